@@ -1,0 +1,370 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle.
+
+Each test checks the oracle against mathematics, a closed form, a library
+routine or brute force on tiny inputs, chosen so that a plausible slip (a
+dropped term, a wrong sign, a swapped axis, an off-by-one in a block edge, a
+wrong tie-break) fails at least one of them.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+
+from oracle import rope, hsa, path
+from oracle.attention import attend
+from cva_workload import WORKLOADS, chunk_inputs, bf16_bits_to_f32
+
+
+RNG = np.random.default_rng(1234)
+
+
+# --- RoPE ------------------------------------------------------------------
+
+def _rot(x, t, h, w):
+    x = np.asarray(x, dtype=np.float64)
+    ang = rope.pair_angles(x.shape[-1], np.atleast_1d(t), np.atleast_1d(h), np.atleast_1d(w))
+    return rope.rotate(x[None, :], ang)[0]
+
+
+def test_rope_closed_form_d6():
+    # D=6: one pair per axis, every rate is 10000**0 = 1, so the angles are the
+    # positions themselves.
+    x = np.array([1.0, 0.0, 0.0, 1.0, 1.0, 1.0])
+    y = _rot(x, 1, 2, 3)
+    c, s = math.cos, math.sin
+    want = [c(1), s(1), -s(2), c(2), c(3) - s(3), s(3) + c(3)]
+    np.testing.assert_allclose(y, want, rtol=0, atol=1e-15)
+
+
+def test_axis_split_matches_wan_sections():
+    # 128 -> 44/42/42 dims, 64 -> 24/20/20 dims (pairs 22/21/21 and 12/10/10).
+    assert rope.axis_split(128) == (22, 21, 21)
+    assert rope.axis_split(64) == (12, 10, 10)
+
+
+def test_rope_rates_first_and_last_pair():
+    # pair j of an axis with p pairs turns at 10000**(-j/p) rad per position
+    for p in (10, 12, 21, 22):
+        f = rope.axis_freqs(p)
+        assert f[0] == 1.0
+        assert f[-1] == pytest.approx(10000.0 ** (-(p - 1) / p), rel=1e-15)
+        assert np.all(np.diff(f) < 0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope_norm_preserved(D):
+    x = RNG.standard_normal((50, D))
+    t, h, w = RNG.integers(0, 300, 50), RNG.integers(0, 45, 50), RNG.integers(0, 80, 50)
+    y = rope.rotate(x, rope.pair_angles(D, t, h, w))
+    nx = x[:, 0::2] ** 2 + x[:, 1::2] ** 2
+    ny = y[:, 0::2] ** 2 + y[:, 1::2] ** 2
+    np.testing.assert_allclose(ny, nx, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope_relative_position(D):
+    # <R(m) q, R(n) k> == <q, R(n - m) k>: scores depend on the offset only.
+    for _ in range(20):
+        q, k = RNG.standard_normal(D), RNG.standard_normal(D)
+        m = RNG.integers(0, 200, 3)
+        n = RNG.integers(0, 200, 3)
+        lhs = _rot(q, *m) @ _rot(k, *n)
+        rhs = q @ _rot(k, *(n - m))
+        assert lhs == pytest.approx(rhs, rel=1e-11, abs=1e-11)
+
+
+def test_rope_position_zero_is_identity():
+    x = RNG.standard_normal((4, 128))
+    y = rope.rotate(x, rope.pair_angles(128, [0] * 4, [0] * 4, [0] * 4))
+    np.testing.assert_array_equal(y, x)
+
+
+def test_rope_axis_sections_in_order_t_h_w():
+    # A coordinate on one axis only moves that axis's section of the vector.
+    D = 128
+    p_t, p_h, p_w = rope.axis_split(D)
+    x = RNG.standard_normal(D)
+    sec = {"t": slice(0, 2 * p_t), "h": slice(2 * p_t, 2 * (p_t + p_h)),
+           "w": slice(2 * (p_t + p_h), D)}
+    for axis, pos in (("t", (5, 0, 0)), ("h", (0, 5, 0)), ("w", (0, 0, 5))):
+        y = _rot(x, *pos)
+        for other, sl in sec.items():
+            if other == axis:
+                assert not np.allclose(y[sl], x[sl])
+            else:
+                np.testing.assert_array_equal(y[sl], x[sl])
+
+
+def test_rope_complex_restatement():
+    # (x0 + i x1) * exp(i phi) with phi built from the pages' t = t0 + f rule.
+    D, Fh, Fw, Fc, t0 = 64, 3, 4, 2, 7
+    x = RNG.standard_normal((1, Fc * Fh * Fw, 1, D))
+    y = rope.rope_chunk(x, Fh, Fw, Fc, t0)[0, :, 0]
+    z = x[0, :, 0, 0::2] + 1j * x[0, :, 0, 1::2]
+    p_t, p_h, p_w = rope.axis_split(D)
+    for n in range(Fc * Fh * Fw):
+        f, r = divmod(n, Fh * Fw)
+        hh, ww = divmod(r, Fw)
+        phi = np.concatenate([(t0 + f) * 10000.0 ** (-np.arange(p_t) / p_t),
+                              hh * 10000.0 ** (-np.arange(p_h) / p_h),
+                              ww * 10000.0 ** (-np.arange(p_w) / p_w)])
+        zz = z[n] * np.exp(1j * phi)
+        np.testing.assert_allclose(y[n, 0::2], zz.real, atol=1e-12)
+        np.testing.assert_allclose(y[n, 1::2], zz.imag, atol=1e-12)
+
+
+def test_global_time_index_tokens():
+    # token n of a chunk starting at s has global t = s + n // T_f
+    t, h, w = rope.token_coords(3, 5, 3, 42)
+    assert list(t[:15]) == [42] * 15 and list(t[15:30]) == [43] * 15 and t[-1] == 44
+    assert h[7] == 1 and w[7] == 2
+
+
+def test_tables_match_direct_angles():
+    (ct, st), (ch, sh), (cw, sw) = rope.tables(128, 240, 30, 52)
+    assert ct.shape == (240, 22) and ch.shape == (30, 21) and cw.shape == (52, 21)
+    ang = rope.pair_angles(128, [239], [29], [51])[0]
+    np.testing.assert_allclose(ct[239], np.cos(ang[:22]), atol=1e-15)
+    np.testing.assert_allclose(sw[51], np.sin(ang[43:]), atol=1e-15)
+
+
+# --- bf16 rounding ------------------------------------------------------------
+
+def test_round_bf16_matches_bit_rounding_of_float32():
+    # For float32-representable inputs the exact rounding equals rounding the
+    # float32 bit pattern (a different construction).
+    from cva_workload import bf16_bits
+    x = RNG.standard_normal(100000).astype(np.float32) * np.float32(3.0)
+    x[:4] = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -0.0, 2 ** -130]   # ties and a subnormal
+    want = bf16_bits_to_f32(bf16_bits(x)).astype(np.float64)
+    got = path.round_bf16(x.astype(np.float64))
+    np.testing.assert_array_equal(got, want)
+
+
+# --- pooling ------------------------------------------------------------------
+
+def test_block_means_ragged_tail_and_weighted_frame_mean():
+    x = RNG.standard_normal((2, 1560, 8))
+    bm = hsa.block_means(x, 64)
+    assert bm.shape == (2, 25, 8)
+    # library mean of the explicit slices, including the 24-token tail
+    np.testing.assert_allclose(bm[:, 24], np.mean(x[:, 1536:1560], axis=1), rtol=1e-13)
+    np.testing.assert_allclose(bm[:, 3], np.mean(x[:, 192:256], axis=1), rtol=1e-13)
+    counts = np.array([64] * 24 + [24])
+    fm = np.average(bm, axis=1, weights=counts)
+    np.testing.assert_allclose(hsa.frame_mean(x), fm, rtol=1e-12, atol=1e-15)
+    # the frame mean is a token mean, not a mean of block means
+    assert not np.allclose(hsa.frame_mean(x), bm.mean(axis=1))
+
+
+def test_pool_queries_layout():
+    B, H, D, Fh, Fw, Fc, blk = 1, 2, 4, 3, 5, 2, 8
+    q = RNG.standard_normal((B, Fc * Fh * Fw, H, D))
+    qb, qf = path.pool_queries(q, Fh * Fw, blk, Fc)
+    assert qb.shape == (B, H, Fc * 2, D)
+    # query block 3 = frame 1, block 1 = tokens 15+8 .. 15+14
+    np.testing.assert_allclose(qb[0, 1, 3], q[0, 23:30, 1].mean(0), rtol=1e-13)
+    np.testing.assert_allclose(qf[0, 0, 1], q[0, 15:30, 0].mean(0), rtol=1e-13)
+
+
+# --- selection ----------------------------------------------------------------
+
+def _brute_topk(scores, k):
+    best = None
+    for sub in itertools.combinations(range(len(scores)), k):
+        key = (sum(scores[i] for i in sub), [-i for i in sub])
+        if best is None or key > best[0]:
+            best = (key, sub)
+    return np.array(best[1])
+
+
+def test_topk_equals_brute_force_with_ties():
+    for trial in range(60):
+        n = int(RNG.integers(1, 10))
+        k = int(RNG.integers(0, n + 1))
+        # small integer scores force ties
+        s = RNG.integers(-3, 4, n).astype(np.float64)
+        got, _ = hsa.topk(s, k)
+        np.testing.assert_array_equal(got, _brute_topk(list(s), k))
+
+
+def test_topk_tie_goes_to_lower_index():
+    got, gap = hsa.topk(np.array([1.0, 2.0, 2.0, 2.0, 0.5]), 2)
+    assert list(got) == [1, 2] and gap == 0.0
+
+
+def test_block_select_ids_and_full_budget():
+    nb, D = 3, 4
+    frames = np.array([2, 5])
+    kb = RNG.standard_normal((2, nb, D))
+    q = RNG.standard_normal(D)
+    ids, gap = hsa.block_select(q, kb, frames, nb, 6)
+    assert list(ids) == [6, 7, 8, 15, 16, 17] and gap == math.inf
+    ids, _ = hsa.block_select(q, kb, frames, nb, 1)
+    sc = np.concatenate([kb[0] @ q, kb[1] @ q])
+    g = [6, 7, 8, 15, 16, 17][int(np.argmax(sc))]
+    assert list(ids) == [g]
+
+
+def test_frame_select_takes_all_when_few():
+    ft, gap = hsa.frame_select(np.ones(4), np.zeros((3, 4)), np.array([0, 1, 2]), 5)
+    assert list(ft) == [0, 1, 2] and gap == math.inf
+
+
+def _c1_path(wl, t_shift=0, store="bf16", dense=None):
+    """Run the c1 workload's chunks 1..4 through the oracle path."""
+    cache = path.FrameCache(wl.B, wl.H, wl.D, wl.T_f, wl.blk, wl.window)
+    out = None
+    for c in range(1, wl.chunk + 1):
+        x = chunk_inputs(wl, c)
+        q, k, v = (bf16_bits_to_f32(x[n]).astype(np.float64) for n in ("q", "k", "v"))
+        t0 = wl.t0_of(c) + t_shift
+        hist_frames = min(wl.t0_of(c), wl.window - wl.Fc)
+        k_f, k_b = hsa.budget(c, hist_frames, wl.nb, dense=wl.dense if dense is None else dense,
+                              k_f_max=wl.k_f_max, k_b_fixed=wl.k_b_fixed,
+                              d_base=wl.d_base, d_slope=wl.d_slope, d_pivot=wl.d_pivot)
+        out = path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0,
+                             k_f=k_f, k_b=k_b, dense=wl.dense if dense is None else dense,
+                             store=store)
+    return cache, out
+
+
+def test_c1_sparse_selection_is_brute_force_top4():
+    # Tiny case, sparse: top-4 of 9 frames, then top-4 of their 4 blocks (all).
+    wl = WORKLOADS["c1s"]
+    cache, out = _c1_path(wl)
+    hist = out["hist"]
+    assert list(hist) == list(range(9))
+    for b in range(wl.B):
+        for h in range(wl.H):
+            for qb in range(wl.NQB):
+                qbar = out["qbar_blk"][b, h, qb]
+                sc = [cache.frames[t]["kf"][b, h] @ qbar for t in hist]
+                want = _brute_topk(sc, 4)                     # C(9,4)=126 subsets
+                assert list(out["frames"][b, h, qb]) == list(hist[want])
+                assert list(out["blocks"][b, h, qb]) == list(hist[want])   # nb = 1
+
+
+# --- attention ------------------------------------------------------------------
+
+def test_attend_special_cases():
+    D = 16
+    k = RNG.standard_normal((10, D))
+    v = RNG.standard_normal((10, D))
+    q = RNG.standard_normal((3, D))
+    # constant V -> that vector
+    cv = np.tile(RNG.standard_normal(D), (10, 1))
+    o, _ = attend(q, k, cv, 0.25)
+    np.testing.assert_allclose(o, cv[:3], rtol=1e-13)
+    # Q = 0 -> mean of V, lse = log(nk)
+    o, lse = attend(np.zeros((2, D)), k, v, 0.25)
+    np.testing.assert_allclose(o, np.tile(v.mean(0), (2, 1)), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(10), rtol=1e-14)
+    # a single key -> its value
+    o, _ = attend(q, k[:1], v[:1], 0.25)
+    np.testing.assert_allclose(o, np.tile(v[0], (3, 1)), rtol=1e-14)
+    # permutation of the keys changes nothing
+    perm = RNG.permutation(10)
+    o1, l1 = attend(q, k, v, 0.25)
+    o2, l2 = attend(q, k[perm], v[perm], 0.25)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12)
+    # library softmax / logsumexp
+    s = 0.25 * q @ k.T
+    np.testing.assert_allclose(o1, scipy.special.softmax(s, axis=1) @ v, rtol=1e-12)
+    np.testing.assert_allclose(l1, scipy.special.logsumexp(s, axis=1), rtol=1e-13)
+
+
+def test_full_budget_sparse_equals_dense_bruteforce():
+    # c1: sparse path at full budget (k_f = 9, k_b = 9) == softmax over the
+    # whole cache, computed by scipy for every query separately.
+    wl = WORKLOADS["c1s"].replace(k_f_max=9, k_b_fixed=9)
+    cache, out = _c1_path(wl)
+    assert out["blocks"].shape[-1] == 9
+    all_t = sorted(cache.frames)
+    scale = 1 / math.sqrt(wl.D)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            K = np.concatenate([cache.frames[t]["k"][b, h] for t in all_t])
+            V = np.concatenate([cache.frames[t]["v"][b, h] for t in all_t])
+            assert K.shape[0] == 12 * 64
+            for n in range(0, wl.Lq, 7):
+                p = scipy.special.softmax(scale * K @ out["q_rot"][b, n, h])
+                np.testing.assert_allclose(out["o"][b, n, h], p @ V, rtol=1e-10, atol=1e-12)
+    # and the dense path gives the same numbers
+    _, outd = _c1_path(WORKLOADS["c1"])
+    np.testing.assert_allclose(outd["o"], out["o"], rtol=1e-12, atol=1e-13)
+
+
+def test_global_shift_leaves_outputs_unchanged():
+    # t0 = 9 and t0 = 109 (history shifted along): identical scores and outputs.
+    for key in ("c1", "c1s"):
+        wl = WORKLOADS[key]
+        _, a = _c1_path(wl, 0, store="f64")
+        _, b = _c1_path(wl, 100, store="f64")
+        np.testing.assert_allclose(a["o"], b["o"], rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(a["lse"], b["lse"], rtol=1e-11)
+        if a["blocks"] is not None:
+            np.testing.assert_array_equal(a["blocks"] % wl.nb, b["blocks"] % wl.nb)
+            np.testing.assert_array_equal(a["frames"] + 100, b["frames"])
+        # the rotated tensors themselves do change with t
+        assert not np.allclose(a["q_rot"], b["q_rot"])
+
+
+def test_unselected_blocks_do_not_matter():
+    wl = WORKLOADS["c1s"]
+    cache, out = _c1_path(wl)
+    b, h, qb = 0, 1, 2
+    chosen = set(int(g) for g in out["blocks"][b, h, qb])
+    other = [t for t in out["hist"] if t not in chosen][0]
+    rows = np.arange(qb * 64, qb * 64 + 64)
+    o1, _ = path.attend_chunk(out["q_rot"], cache, wl.t0, wl.Fc, out["blocks"], rows)
+    cache.frames[other]["v"][b, h] += 100.0
+    o2, _ = path.attend_chunk(out["q_rot"], cache, wl.t0, wl.Fc, out["blocks"], rows)
+    np.testing.assert_array_equal(o1[b, rows, h], o2[b, rows, h])
+    cache.frames[min(chosen)]["v"][b, h] += 100.0
+    o3, _ = path.attend_chunk(out["q_rot"], cache, wl.t0, wl.Fc, out["blocks"], rows)
+    assert not np.allclose(o1[b, rows, h], o3[b, rows, h])
+
+
+def test_rolling_window_evicts_and_history_range():
+    c = path.FrameCache(1, 1, 4, 2, 2, window=5)
+    for t0 in (0, 2, 4):
+        c.append(np.zeros((1, 4, 1, 4)), np.zeros((1, 4, 1, 4)), t0, 2)
+    assert sorted(c.frames) == [1, 2, 3, 4, 5]
+    assert list(c.history(4, 2)) == [1, 2, 3]
+
+
+# --- chunk budget ------------------------------------------------------------------
+
+def _b(wl, chunk, hist):
+    return hsa.budget(chunk, hist, wl.nb, dense=wl.dense, k_f_max=wl.k_f_max,
+                      d_base=wl.d_base, d_slope=wl.d_slope, d_pivot=wl.d_pivot,
+                      k_b_fixed=wl.k_b_fixed)
+
+
+def test_cag_literal_schedule_integers():
+    # s_i = 3/4 - (i-6)/60 -> density (9+i)/60 of 3(i-1)*25 history blocks,
+    # rounded half up: 11/60*75=13.75->14, 12/60*150=30, 13/60*225=48.75->49,
+    # 14/60*300=70, 15/60*375=93.75->94, 16/60*450=120.
+    wl = WORKLOADS["c3"]
+    got = [_b(wl, i, 3 * (i - 1)) for i in range(1, 8)]
+    assert got == [(0, 0), (3, 14), (6, 30), (8, 49), (8, 70), (8, 94), (8, 120)]
+    assert hsa.density(wl.d_base, wl.d_slope, wl.d_pivot, 7) == Fraction(16, 60)
+
+
+def test_cag_mirrored_schedule_integers():
+    # density (21-i)/60: 19/60*75=23.75->24, 45, 63.75->64, 80, 93.75->94, 105
+    wl = WORKLOADS["c3"].replace(d_slope=Fraction(-1, 60))
+    got = [_b(wl, i, 3 * (i - 1))[1] for i in range(2, 8)]
+    assert got == [24, 45, 64, 80, 94, 105]
+
+
+def test_cag_other_workloads():
+    assert _b(WORKLOADS["c4"], 7, 18) == (6, 104)          # 0.2*522 = 104.4
+    assert _b(WORKLOADS["c5"], 80, 57) == (20, 285)        # 0.2*1425
+    assert _b(WORKLOADS["c5"], 2, 3) == (3, 15)
+    assert _b(WORKLOADS["c2"], 7, 18) == (18, 450)         # dense
+    assert _b(WORKLOADS["c1s"], 4, 9) == (4, 4)
