@@ -1,0 +1,579 @@
+// C ABI of libcva: argument checks, workspace and cache layout, and the
+// launch sequence of the per-chunk path. Nothing here allocates device
+// memory or synchronises (except cva_device_status, which reads the device
+// error word).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+
+using namespace cva;
+
+namespace {
+
+thread_local char g_msg[512] = "";
+thread_local cudaEvent_t g_stage_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+thread_local bool g_stage_on = false;
+
+cudaError_t stage_mark(int i, cudaStream_t s) {
+  return g_stage_on ? cudaEventRecord(g_stage_ev[i], s) : cudaSuccess;
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(CVA_ELAUNCH, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Device error word, one per device; kernels receive its address.
+__device__ int g_dev_err;
+
+int* device_error_word() {
+  static std::mutex mu;
+  static int* ptrs[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(const cva_shape* s) {
+  if (!s) return fail(CVA_EINVAL, "shape is NULL");
+  if (s->batch < 1 || s->heads < 1 || s->frame_h < 1 || s->frame_w < 1 || s->chunk_frames < 1)
+    return fail(CVA_EINVAL, "shape: batch, heads, frame_h, frame_w, chunk_frames must be >= 1");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(CVA_ENOTSUP, "head_dim %d not supported (64 or 128)", s->head_dim);
+  if (s->block != 64 && s->block != 128)
+    return fail(CVA_ENOTSUP, "block %d not supported (64 or 128)", s->block);
+  if ((int64_t)s->batch * s->heads > 65535) return fail(CVA_ENOTSUP, "batch*heads > 65535");
+  const int64_t tf = (int64_t)s->frame_h * s->frame_w;
+  if (tf > (1 << 20)) return fail(CVA_ENOTSUP, "tokens per frame > 2^20");
+  const Dims d = make_dims(*s);
+  if ((int64_t)d.Fc * d.nb > 65535) return fail(CVA_ENOTSUP, "chunk_frames * blocks per frame > 65535");
+  return CVA_OK;
+}
+
+bool same_shape(const cva_shape& a, const cva_shape& b) {
+  return a.batch == b.batch && a.heads == b.heads && a.head_dim == b.head_dim &&
+         a.frame_h == b.frame_h && a.frame_w == b.frame_w && a.chunk_frames == b.chunk_frames &&
+         a.block == b.block;
+}
+
+int check_cache(const cva_kv_cache* c) {
+  if (!c) return fail(CVA_EINVAL, "cache is NULL");
+  int rc = check_shape(&c->shape);
+  if (rc) return rc;
+  if (!c->k || !c->v || !c->kpool_blk || !c->kpool_frm)
+    return fail(CVA_EINVAL, "cache has a NULL buffer");
+  if (!aligned(c->k, 256) || !aligned(c->v, 256) || !aligned(c->kpool_blk, 16) ||
+      !aligned(c->kpool_frm, 16))
+    return fail(CVA_EINVAL, "cache buffers must be 256-byte (k, v) and 16-byte (pools) aligned");
+  if (c->window < c->shape.chunk_frames)
+    return fail(CVA_EINVAL, "cache window %d < chunk_frames %d", c->window, c->shape.chunk_frames);
+  const Dims d = make_dims(c->shape);
+  if ((int64_t)c->window * d.T_pad / 64 >= 65536)
+    return fail(CVA_ENOTSUP, "window * padded frame rows too large (>= 2^22 rows)");
+  return CVA_OK;
+}
+
+int check_tables(const cva_rope_tables* t, const Dims& d, int t0) {
+  if (!t) return fail(CVA_EINVAL, "rope tables are NULL");
+  if (!t->cos_t || !t->sin_t || !t->cos_h || !t->sin_h || !t->cos_w || !t->sin_w)
+    return fail(CVA_EINVAL, "rope tables have a NULL pointer");
+  if (t->head_dim != d.D) return fail(CVA_EINVAL, "rope tables built for head_dim %d, shape has %d", t->head_dim, d.D);
+  if (t->frame_h < d.Fh || t->frame_w < d.Fw)
+    return fail(CVA_ERANGE, "rope tables cover %dx%d positions, frame is %dx%d", t->frame_h, t->frame_w, d.Fh, d.Fw);
+  if (t0 < 0 || (int64_t)t0 + d.Fc > t->max_t)
+    return fail(CVA_ERANGE, "global time %d..%d outside the temporal table (max_t %d)", t0, t0 + d.Fc - 1, t->max_t);
+  return CVA_OK;
+}
+
+RopeTab make_tab(const cva_rope_tables* t, int D) {
+  RopeTab r;
+  r.cos_t = t->cos_t; r.sin_t = t->sin_t; r.cos_h = t->cos_h; r.sin_h = t->sin_h;
+  r.cos_w = t->cos_w; r.sin_w = t->sin_w;
+  axis_pairs(D, &r.pt, &r.ph, &r.pw);
+  return r;
+}
+
+// History frames [t_lo, t_lo + F) a chunk at t0 sees.
+void history(const cva_kv_cache* c, int t0, int* t_lo, int* F) {
+  int lo = t0 + c->shape.chunk_frames - c->window;
+  if (lo < c->t_begin) lo = c->t_begin;
+  *t_lo = lo;
+  *F = t0 > lo ? t0 - lo : 0;
+}
+
+struct ChunkWs {
+  size_t q_rot, qpool, frame_idx, block_idx, block_cnt, total;
+};
+
+ChunkWs chunk_ws_layout(const Dims& d, int k_f, int k_b) {
+  ChunkWs w;
+  const size_t bhq = (size_t)d.B * d.H * d.NQB;
+  size_t off = 0;
+  w.q_rot = off; off += round256((size_t)d.B * d.H * d.Fc * d.T_pad * d.D * 2);
+  w.qpool = off; off += round256(bhq * d.D * 4);
+  w.frame_idx = off; off += round256(bhq * (size_t)(k_f > 0 ? k_f : 0) * 4);
+  w.block_idx = off; off += round256(bhq * (size_t)(k_b > 0 ? k_b : 0) * 4);
+  w.block_cnt = off; off += round256(bhq * 4);
+  w.total = off;
+  return w;
+}
+
+int check_attn_limits(const Dims& d, int F, bool dense, int k_b_max) {
+  const int upb = d.blk / 64;
+  const int64_t cur = (int64_t)d.Fc * d.nb * upb;
+  int64_t hist;
+  if (dense) {
+    hist = (int64_t)F * d.nb * upb;
+  } else {
+    if ((int64_t)F * d.nb > 32 * kAttnMaxBitmapWords)
+      return fail(CVA_ENOTSUP, "history blocks %lld exceed %d for the sparse attention",
+                  (long long)F * d.nb, 32 * kAttnMaxBitmapWords);
+    const int nq = d.blk == 64 ? 2 : 1;
+    int64_t u = (int64_t)nq * k_b_max;
+    if (u > (int64_t)F * d.nb) u = (int64_t)F * d.nb;
+    hist = u * upb;
+  }
+  if (hist + cur > kAttnMaxEntries)
+    return fail(CVA_ENOTSUP, "key units per query tile %lld exceed %d", (long long)(hist + cur),
+                kAttnMaxEntries);
+  return CVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cva_version(void) { return CVA_VERSION; }
+
+const char* cva_last_error(void) { return g_msg; }
+
+int cva_device_status(int32_t* code, int32_t clear) {
+  if (!code) return fail(CVA_EINVAL, "code is NULL");
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_dev_err, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  *code = v;
+  if (clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  return CVA_OK;
+}
+
+int cva_set_stage_events(void* const* events, int32_t n) {
+  if (n == 0 && events == nullptr) {
+    g_stage_on = false;
+    return CVA_OK;
+  }
+  if (n != 4 || !events) return fail(CVA_EINVAL, "stage events: pass 4 events, or NULL and 0");
+  for (int i = 0; i < 4; ++i) {
+    if (!events[i]) return fail(CVA_EINVAL, "stage event %d is NULL", i);
+    g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_stage_on = true;
+  return CVA_OK;
+}
+
+int cva_rope_axis_pairs(int32_t head_dim, int32_t* p_t, int32_t* p_h, int32_t* p_w) {
+  if (!p_t || !p_h || !p_w) return fail(CVA_EINVAL, "NULL output");
+  if (head_dim < 6 || head_dim % 2) return fail(CVA_EINVAL, "head_dim must be even and >= 6");
+  int a, b, c;
+  axis_pairs(head_dim, &a, &b, &c);
+  *p_t = a; *p_h = b; *p_w = c;
+  return CVA_OK;
+}
+
+int cva_rope3d_precompute(const cva_rope_cfg* cfg, float* cos_t, float* sin_t, float* cos_h,
+                          float* sin_h, float* cos_w, float* sin_w) {
+  if (!cfg) return fail(CVA_EINVAL, "cfg is NULL");
+  if (!cos_t || !sin_t || !cos_h || !sin_h || !cos_w || !sin_w) return fail(CVA_EINVAL, "NULL table");
+  if (cfg->head_dim < 6 || cfg->head_dim % 2) return fail(CVA_EINVAL, "head_dim must be even and >= 6");
+  if (cfg->max_t < 1 || cfg->frame_h < 1 || cfg->frame_w < 1) return fail(CVA_EINVAL, "table rows must be >= 1");
+  if (!(cfg->theta > 1.0)) return fail(CVA_EINVAL, "theta must be > 1");
+  int p[3];
+  axis_pairs(cfg->head_dim, &p[0], &p[1], &p[2]);
+  const int rows[3] = {cfg->max_t, cfg->frame_h, cfg->frame_w};
+  float* cs[3] = {cos_t, cos_h, cos_w};
+  float* sn[3] = {sin_t, sin_h, sin_w};
+  for (int a = 0; a < 3; ++a) {
+    for (int pos = 0; pos < rows[a]; ++pos) {
+      for (int j = 0; j < p[a]; ++j) {
+        // rate theta^(-2j / (2 p_a)) radians per unit of position
+        const double rate = pow(cfg->theta, -(2.0 * j) / (2.0 * p[a]));
+        const double ang = (double)pos * rate;
+        cs[a][(size_t)pos * p[a] + j] = (float)cos(ang);
+        sn[a][(size_t)pos * p[a] + j] = (float)sin(ang);
+      }
+    }
+  }
+  return CVA_OK;
+}
+
+int cva_history_frames(const cva_kv_cache* cache, int32_t t0, int32_t* t_lo, int32_t* count) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!t_lo || !count) return fail(CVA_EINVAL, "NULL output");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  int lo, F;
+  history(cache, t0, &lo, &F);
+  *t_lo = lo;
+  *count = F;
+  return CVA_OK;
+}
+
+int cva_kv_cache_bytes(const cva_shape* shape, int32_t window, size_t* bytes) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!bytes) return fail(CVA_EINVAL, "bytes is NULL");
+  if (window < shape->chunk_frames) return fail(CVA_EINVAL, "window < chunk_frames");
+  const Dims d = make_dims(*shape);
+  const size_t slots = (size_t)d.B * d.H * window;
+  *bytes = 2 * round256(slots * d.T_pad * d.D * 2) + round256(slots * d.nb * d.D * 4) +
+           round256(slots * d.D * 4);
+  return CVA_OK;
+}
+
+int cva_kv_cache_init(cva_kv_cache* cache, void* dev_mem, size_t bytes, const cva_shape* shape,
+                      int32_t window, int32_t t_begin) {
+  if (!cache || !dev_mem) return fail(CVA_EINVAL, "NULL cache or memory");
+  size_t need = 0;
+  int rc = cva_kv_cache_bytes(shape, window, &need);
+  if (rc) return rc;
+  if (bytes < need) return fail(CVA_ENOMEM, "cache arena %zu bytes < %zu needed", bytes, need);
+  if (!aligned(dev_mem, 256)) return fail(CVA_EINVAL, "cache arena must be 256-byte aligned");
+  if (t_begin < 0) return fail(CVA_EINVAL, "t_begin < 0");
+  const Dims d = make_dims(*shape);
+  const size_t slots = (size_t)d.B * d.H * window;
+  char* p = static_cast<char*>(dev_mem);
+  cache->k = p; p += round256(slots * d.T_pad * d.D * 2);
+  cache->v = p; p += round256(slots * d.T_pad * d.D * 2);
+  cache->kpool_blk = reinterpret_cast<float*>(p); p += round256(slots * d.nb * d.D * 4);
+  cache->kpool_frm = reinterpret_cast<float*>(p);
+  cache->window = window;
+  cache->t_begin = t_begin;
+  cache->shape = *shape;
+  return check_cache(cache);
+}
+
+int cva_cag_budget(const cva_cag_cfg* cfg, int32_t chunk_index, int32_t hist_frames,
+                   int32_t blocks_per_frame, int32_t* k_f, int32_t* k_b) {
+  if (!cfg || !k_f || !k_b) return fail(CVA_EINVAL, "NULL argument");
+  if (chunk_index < 1 || hist_frames < 0 || blocks_per_frame < 1)
+    return fail(CVA_EINVAL, "chunk_index >= 1, hist_frames >= 0, blocks_per_frame >= 1 required");
+  const int64_t all = (int64_t)hist_frames * blocks_per_frame;
+  if (cfg->dense || chunk_index <= 1 || hist_frames == 0) {
+    *k_f = hist_frames;
+    *k_b = (int32_t)all;
+    return CVA_OK;
+  }
+  if (cfg->k_f_max < 1) return fail(CVA_EINVAL, "k_f_max must be >= 1");
+  const int kf = cfg->k_f_max < hist_frames ? cfg->k_f_max : hist_frames;
+  const int64_t cand = (int64_t)kf * blocks_per_frame;
+  int64_t kb;
+  if (cfg->k_b_fixed >= 0) {
+    kb = cfg->k_b_fixed;
+  } else {
+    if (cfg->d_base_den <= 0 || cfg->d_slope_den <= 0) return fail(CVA_EINVAL, "denominators must be > 0");
+    // d = d_base + d_slope * (i - pivot) as one fraction num/den (exact)
+    const int64_t den = cfg->d_base_den * cfg->d_slope_den;
+    int64_t num = cfg->d_base_num * cfg->d_slope_den +
+                  cfg->d_slope_num * cfg->d_base_den * (int64_t)(chunk_index - cfg->pivot);
+    if (num < 0) num = 0;
+    if (num > den) num = den;
+    // floor(d * all + 1/2) = floor((2 * num * all + den) / (2 * den))
+    kb = (2 * num * all + den) / (2 * den);
+  }
+  if (kb > cand) kb = cand;
+  *k_f = kf;
+  *k_b = (int32_t)kb;
+  return CVA_OK;
+}
+
+int cva_rope3d_apply(const void* x, void* y, const cva_rope_tables* tables, const cva_shape* shape,
+                     int32_t t0, int32_t out_layout, cva_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!x || !y) return fail(CVA_EINVAL, "x or y is NULL");
+  if (!aligned(x, 16) || !aligned(y, 16)) return fail(CVA_EINVAL, "x and y must be 16-byte aligned");
+  if (out_layout != 0 && out_layout != 1) return fail(CVA_EINVAL, "out_layout must be 0 or 1");
+  const Dims d = make_dims(*shape);
+  rc = check_tables(tables, d, t0);
+  if (rc) return rc;
+  RopePoolArgs a = {};
+  a.job[0] = {static_cast<const uint16_t*>(x), kTokenMajor, static_cast<uint16_t*>(y),
+              out_layout == 0 ? (int)kTokenMajor : (int)kHeadMajor, 1, nullptr, kPoolNone};
+  a.njobs = 1;
+  a.tab = make_tab(tables, d.D);
+  a.d = d;
+  a.t0 = t0;
+  a.W = 1;
+  cudaError_t e = launch_rope_pool(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "rope3d_apply launch");
+}
+
+int cva_kv_append(const void* k, const void* v, const cva_kv_cache* cache,
+                  const cva_rope_tables* tables, int32_t t0, cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!k || !v) return fail(CVA_EINVAL, "k or v is NULL");
+  if (!aligned(k, 16) || !aligned(v, 16)) return fail(CVA_EINVAL, "k and v must be 16-byte aligned");
+  const Dims d = make_dims(cache->shape);
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  if (tables) {
+    rc = check_tables(tables, d, t0);
+    if (rc) return rc;
+  }
+  RopePoolArgs a = {};
+  a.job[0] = {static_cast<const uint16_t*>(k), kTokenMajor, static_cast<uint16_t*>(cache->k),
+              kCacheSlots, tables ? 1 : 0, cache->kpool_blk, kPoolCache};
+  a.job[1] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
+              kCacheSlots, 0, nullptr, kPoolNone};
+  a.njobs = 2;
+  if (tables) a.tab = make_tab(tables, d.D);
+  else axis_pairs(d.D, &a.tab.pt, &a.tab.ph, &a.tab.pw);
+  a.d = d;
+  a.t0 = t0;
+  a.W = cache->window;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rope_pool(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
+  e = launch_frame_pool(fp, s);
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "kv_append frame pool launch");
+}
+
+int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk, float* qpool_frm,
+                     cva_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q_rot || !qpool_blk) return fail(CVA_EINVAL, "q_rot or qpool_blk is NULL");
+  if (!aligned(q_rot, 16)) return fail(CVA_EINVAL, "q_rot must be 16-byte aligned");
+  const Dims d = make_dims(*shape);
+  RopePoolArgs a = {};
+  a.job[0] = {static_cast<const uint16_t*>(q_rot), kHeadMajor, nullptr, kHeadMajor, 0, qpool_blk,
+              kPoolChunk};
+  a.njobs = 1;
+  axis_pairs(d.D, &a.tab.pt, &a.tab.ph, &a.tab.pw);
+  a.d = d;
+  a.t0 = 0;
+  a.W = 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rope_pool(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "hsa_compress launch");
+  if (qpool_frm) {
+    FramePoolArgs fp = {qpool_blk, qpool_frm, kPoolChunk, d, 0, 1};
+    e = launch_frame_pool(fp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "hsa_compress frame pool launch");
+  }
+  return CVA_OK;
+}
+
+static int select_impl(const float* qpool_blk, const cva_kv_cache* cache, int t0, int k_f, int k_b,
+                       int32_t* frame_idx, int32_t* block_idx, int32_t* block_cnt, int k_b_max,
+                       cudaStream_t s) {
+  const Dims d = make_dims(cache->shape);
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
+  const int kfe = k_f < F ? k_f : F;
+  if (F > 0 && k_f < 1) return fail(CVA_ERANGE, "k_f must be >= 1 when there is history");
+  if (k_b < 0 || (int64_t)k_b > (int64_t)kfe * d.nb)
+    return fail(CVA_ERANGE, "k_b %d outside [0, %d] (k_f_eff * blocks per frame)", k_b, kfe * d.nb);
+  if (F > 256) return fail(CVA_ENOTSUP, "history frames %d > 256", F);
+  if ((int64_t)kfe * d.nb > 1024) return fail(CVA_ENOTSUP, "candidate blocks %d > 1024", kfe * d.nb);
+  SelectArgs a = {};
+  a.qpool = qpool_blk;
+  a.kpool_blk = cache->kpool_blk;
+  a.kpool_frm = cache->kpool_frm;
+  a.frame_idx = frame_idx;
+  a.block_idx = block_idx;
+  a.block_cnt = block_cnt;
+  a.d = d;
+  a.W = cache->window;
+  a.t_lo = t_lo;
+  a.F = F;
+  a.k_f = kfe;
+  a.k_b = k_b;
+  a.k_f_stride = kfe;
+  a.k_b_max = k_b_max;
+  if (F == 0) {
+    // Nothing to pick: every count is zero.
+    if (block_cnt) {
+      cudaError_t e = cudaMemsetAsync(block_cnt, 0, (size_t)d.B * d.H * d.NQB * 4, s);
+      if (e != cudaSuccess) return cuda_fail(e, "hsa_select memset");
+    }
+    return CVA_OK;
+  }
+  cudaError_t e = launch_select(a, s);
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "hsa_select launch");
+}
+
+int cva_hsa_select(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0, int32_t k_f,
+                   int32_t k_b, int32_t* frame_idx, int32_t* block_idx, int32_t* block_cnt,
+                   cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!qpool_blk || !block_idx || !block_cnt) return fail(CVA_EINVAL, "NULL buffer");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  return select_impl(qpool_blk, cache, t0, k_f, k_b, frame_idx, block_idx, block_cnt, k_b,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int cva_attn_workspace_bytes(const cva_shape* shape, int32_t k_b_max, size_t* bytes) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!bytes) return fail(CVA_EINVAL, "bytes is NULL");
+  (void)k_b_max;
+  *bytes = 0;
+  return CVA_OK;
+}
+
+static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const int32_t* block_idx,
+                     const int32_t* block_cnt, int k_b_max, void* out, float* lse, cudaStream_t s) {
+  const Dims d = make_dims(cache->shape);
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
+  int rc = check_attn_limits(d, F, block_idx == nullptr, k_b_max);
+  if (rc) return rc;
+  AttnArgs a = {};
+  a.block_idx = block_idx;
+  a.block_cnt = block_cnt;
+  a.k_b_max = k_b_max;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.err = device_error_word();
+  a.d = d;
+  a.W = cache->window;
+  a.t0 = t0;
+  a.t_lo = t_lo;
+  a.F = F;
+  a.MT = (d.Fc * d.T_pad + 127) / 128;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d.D));
+  const char* why = "";
+  cudaError_t e = launch_attention(a, q_rot, cache->k, cache->v, s, &why);
+  if (e == cudaErrorInvalidValue && why[0]) return fail(CVA_ELAUNCH, "attention: %s", why);
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "blocksparse_attn_fwd launch");
+}
+
+int cva_blocksparse_attn_fwd(const void* q_rot, const cva_kv_cache* cache, int32_t t0,
+                             const int32_t* block_idx, const int32_t* block_cnt, int32_t k_b_max,
+                             void* out, float* lse, void* workspace, size_t ws_bytes,
+                             cva_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!q_rot || !out) return fail(CVA_EINVAL, "q_rot or out is NULL");
+  if (!aligned(q_rot, 16) || !aligned(out, 16)) return fail(CVA_EINVAL, "q_rot and out must be 16-byte aligned");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  if (block_idx && (!block_cnt || k_b_max < 0)) return fail(CVA_EINVAL, "sparse call needs block_cnt and k_b_max >= 0");
+  return attn_impl(q_rot, cache, t0, block_idx, block_cnt, block_idx ? k_b_max : 0, out, lse,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, size_t* bytes) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!bytes) return fail(CVA_EINVAL, "bytes is NULL");
+  const Dims d = make_dims(*shape);
+  *bytes = chunk_ws_layout(d, k_f, k_b).total;
+  return CVA_OK;
+}
+
+int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                        const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                        void* workspace, size_t ws_bytes, void* out, float* lse,
+                        cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !workspace) return fail(CVA_EINVAL, "NULL buffer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+    return fail(CVA_EINVAL, "q, k, v, out must be 16-byte and workspace 256-byte aligned");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  const Dims d = make_dims(cache->shape);
+  rc = check_tables(tables, d, t0);
+  if (rc) return rc;
+  const bool dense = k_f < 0;
+  const ChunkWs w = chunk_ws_layout(d, dense ? 0 : k_f, dense ? 0 : k_b);
+  if (ws_bytes < w.total) return fail(CVA_ENOMEM, "workspace %zu bytes < %zu needed", ws_bytes, w.total);
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
+  if (!dense) {
+    const int kfe = k_f < F ? k_f : F;
+    if (F > 0 && k_f < 1) return fail(CVA_ERANGE, "k_f must be >= 1 when there is history");
+    if (k_b < 0 || (int64_t)k_b > (int64_t)kfe * d.nb)
+      return fail(CVA_ERANGE, "k_b %d outside [0, %d] (k_f_eff * blocks per frame)", k_b, kfe * d.nb);
+    if (F > 256) return fail(CVA_ENOTSUP, "history frames %d > 256", F);
+    if ((int64_t)kfe * d.nb > 1024) return fail(CVA_ENOTSUP, "candidate blocks %d > 1024", kfe * d.nb);
+  }
+  rc = check_attn_limits(d, F, dense || F == 0, dense ? 0 : k_b);
+  if (rc) return rc;
+
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws + w.q_rot);
+  float* qpool = reinterpret_cast<float*>(ws + w.qpool);
+  int32_t* fidx = reinterpret_cast<int32_t*>(ws + w.frame_idx);
+  int32_t* bidx = reinterpret_cast<int32_t*>(ws + w.block_idx);
+  int32_t* bcnt = reinterpret_cast<int32_t*>(ws + w.block_cnt);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // steps 1-3: rotate Q (+ block pools) and K (+ append, block pools), copy V
+  RopePoolArgs a = {};
+  a.job[0] = {static_cast<const uint16_t*>(q), kTokenMajor, q_rot, kHeadMajor, 1,
+              dense ? nullptr : qpool, dense ? (int)kPoolNone : (int)kPoolChunk};
+  a.job[1] = {static_cast<const uint16_t*>(k), kTokenMajor, static_cast<uint16_t*>(cache->k),
+              kCacheSlots, 1, cache->kpool_blk, kPoolCache};
+  a.job[2] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
+              kCacheSlots, 0, nullptr, kPoolNone};
+  a.njobs = 3;
+  a.tab = make_tab(tables, d.D);
+  a.d = d;
+  a.t0 = t0;
+  a.W = cache->window;
+  cudaError_t e = stage_mark(0, s);
+  if (e != cudaSuccess) return cuda_fail(e, "stage event");
+  e = launch_rope_pool(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention rope/append launch");
+  FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
+  e = launch_frame_pool(fp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention frame pool launch");
+  if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+
+  // step 4
+  const bool sparse = !dense && F > 0;
+  if (sparse) {
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, s);
+    if (rc) return rc;
+  }
+  if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  // step 5
+  rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
+                 sparse ? k_b : 0, out, lse, s);
+  if (rc) return rc;
+  if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  return CVA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,487 @@
+// Step 5 of the per-chunk path: block-sparse flash attention on sm_100a.
+//
+// "Light Forcing", section 2.2 (execution): attention runs only over the
+// picked frame-block pairs, here together with every token of the current
+// chunk; its cost is independent of how long the history is.
+//
+// One CTA computes a 128-row query tile of one (batch, head). Its key set
+// is a list of 64-row key units in smem: the union of the picked history
+// blocks of the tile's query blocks (two 64-token query blocks share a tile
+// when blk = 64; a unit carries a 2-bit mask of the query blocks that
+// picked it) followed by the current chunk's blocks. Pairs of units form
+// 128-key tiles.
+//
+// Roles (192 threads):
+//   warp 4 (one lane): TMA producer. Q once; then K and V of each key tile,
+//     gathered by block index with one 64-row box per unit and 64-column
+//     chunk, 128-byte swizzle, into a 2-stage ring. No multicast.
+//   warp 5 (one lane): tcgen05.mma issuer. S(n) = Q K(n)^T into one of two
+//     128-column fp32 TMEM buffers; O += P(n) V(n) with P read from TMEM
+//     (bf16, aliased onto the S buffer) and O in TMEM.
+//   warps 0-3: softmax; thread i owns query row i (TMEM lane i): masks,
+//     online max/sum in fp32 (exp2 domain), rescales O in TMEM when the
+//     running max moves, writes P, and finally normalises O into bf16.
+// Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
+// roles leave their loops, in-flight copies and MMAs are drained with a
+// bounded wait and the tensor memory is released.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "kernels.cuh"
+
+namespace cva {
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kAttnThreads = 192;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B: one 64-column chunk
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;  // a Q, K or V tile
+  static constexpr int kQ = 0;
+  static constexpr int kKV = kQ + kTileBytes;  // stage s: K at kKV + 2*s*tile, V after it
+  static constexpr int kEnt = kKV + kStages * 2 * kTileBytes;
+  static constexpr int kBm = kEnt + kAttnMaxEntries * 4;
+  static constexpr int kScan = kBm + 2 * kAttnMaxBitmapWords * 4;
+  static constexpr int kBar = kScan + kAttnMaxBitmapWords * 4;
+  static constexpr int kMisc = kBar + 16 * 8;
+  static constexpr int kBytes = kMisc + 64;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
+};
+
+// Barrier slots.
+enum : int { kBarQ = 0, kBarKVFull = 1, kBarKVEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarO = 9,
+             kBarDrain = 10 };
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// A wait with its own limit that ignores the abort flag (used while draining).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) return;  // 200 ms
+  }
+}
+
+// Key unit: (row64 << 16) | (valid << 8) | mask. row64 indexes 64-row
+// groups inside one (batch, head) slice of the cache.
+__device__ __forceinline__ uint32_t make_unit(int row64, int valid, uint32_t mask) {
+  return ((uint32_t)row64 << 16) | ((uint32_t)valid << 8) | mask;
+}
+
+__device__ __forceinline__ int unit_valid(int block_valid, int u) {
+  int v = block_valid - 64 * u;
+  return v < 0 ? 0 : (v > 64 ? 64 : v);
+}
+
+// Builds the tile's key-unit list in smem; returns the number of units.
+// Must be called by all threads of the CTA.
+__device__ int build_units(const AttnArgs& a, int m, int bh, uint32_t* ents, uint32_t* bm,
+                           uint32_t* wcnt, int* total_slot) {
+  const Dims& d = a.d;
+  const int tid = threadIdx.x;
+  const int upb = d.blk / 64;
+  const int rows64_slot = d.T_pad / 64;
+  int hist = 0;
+  if (a.F > 0) {
+    if (a.block_idx == nullptr) {
+      hist = a.F * d.nb * upb;
+      for (int i = tid; i < hist; i += kAttnThreads) {
+        const int br = i / upb, u = i - br * upb;
+        const int fp = br / d.nb, j = br - fp * d.nb;
+        const int slot = (a.t_lo + fp) % a.W;
+        const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+        ents[i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 3u);
+      }
+    } else {
+      const int nbits = a.F * d.nb;
+      const int nw = (nbits + 31) >> 5;
+      for (int i = tid; i < nw; i += kAttnThreads) {
+        bm[i] = 0u;
+        bm[kAttnMaxBitmapWords + i] = 0u;
+      }
+      __syncthreads();
+      const int nq = (d.blk == 64) ? 2 : 1;
+      for (int q = 0; q < nq; ++q) {
+        const int qb = (d.blk == 64) ? 2 * m + q : m;
+        if (qb >= d.NQB) continue;
+        const size_t u = (size_t)bh * d.NQB + qb;
+        int cnt = a.block_cnt ? a.block_cnt[u] : a.k_b_max;
+        if (cnt < 0 || cnt > a.k_b_max) {
+          if (tid == 0) latch_error(a.err, CVA_DEV_BAD_COUNT);
+          cnt = cnt < 0 ? 0 : a.k_b_max;
+        }
+        const int32_t* lst = a.block_idx + u * a.k_b_max;
+        for (int i = tid; i < cnt; i += kAttnThreads) {
+          const int id = lst[i];
+          const int rel = id - a.t_lo * d.nb;
+          if (id < 0 || rel < 0 || rel >= nbits) {
+            latch_error(a.err, CVA_DEV_BAD_INDEX);
+            continue;
+          }
+          atomicOr(&bm[q * kAttnMaxBitmapWords + (rel >> 5)], 1u << (rel & 31));
+        }
+      }
+      __syncthreads();
+      for (int w = tid; w < nw; w += kAttnThreads)
+        wcnt[w] = __popc(bm[w] | bm[kAttnMaxBitmapWords + w]) * upb;
+      __syncthreads();
+      if (tid < 32) {  // exclusive scan of the per-word counts
+        int carry = 0;
+        for (int base = 0; base < nw; base += 32) {
+          const int w = base + tid;
+          const int v = (w < nw) ? (int)wcnt[w] : 0;
+          int incl = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (tid >= o) incl += t;
+          }
+          if (w < nw) wcnt[w] = (uint32_t)(carry + incl - v);
+          carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (tid == 0) *total_slot = carry;
+      }
+      __syncthreads();
+      hist = *total_slot;
+      for (int w = tid; w < nw; w += kAttnThreads) {
+        const uint32_t b0 = bm[w], b1 = bm[kAttnMaxBitmapWords + w];
+        uint32_t any = b0 | b1;
+        int pos = (int)wcnt[w];
+        while (any) {
+          const int bit = __ffs(any) - 1;
+          any &= any - 1u;
+          const int rel = w * 32 + bit;
+          const int fp = rel / d.nb, j = rel - fp * d.nb;
+          const int slot = (a.t_lo + fp) % a.W;
+          const uint32_t mask =
+              (d.blk == 64) ? (((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1)) : 3u;
+          const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+          for (int u = 0; u < upb; ++u)
+            ents[pos++] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
+        }
+      }
+    }
+  }
+  const int cur = d.Fc * d.nb * upb;
+  for (int i = tid; i < cur; i += kAttnThreads) {
+    const int br = i / upb, u = i - br * upb;
+    const int f = br / d.nb, j = br - f * d.nb;
+    const int slot = (a.t0 + f) % a.W;
+    const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+    ents[hist + i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 3u);
+  }
+  __syncthreads();
+  return hist + cur;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using L = AttnSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int m = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  int* total_slot = reinterpret_cast<int*>(smem + L::kMisc + 8);
+
+  if (tid == 0) {
+    mbar_init(&bar[kBarQ], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar[kBarKVFull + s], 1);
+      mbar_init(&bar[kBarKVEmpty + s], 1);
+      mbar_init(&bar[kBarSFull + s], 1);
+      mbar_init(&bar[kBarPFull + s], 128);
+    }
+    mbar_init(&bar[kBarO], 1);
+    mbar_init(&bar[kBarDrain], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  const int E = build_units(a, m, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
+                            reinterpret_cast<uint32_t*>(smem + L::kScan), total_slot);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int N = (E + 1) >> 1;  // 128-key tiles
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
+      int issued = 0;
+      for (int n = 0; n < N; ++n) {
+        const int st = n & 1;
+        if (n >= 2 && !mbar_wait(&bar[kBarKVEmpty + st], ((n - 2) >> 1) & 1, abort_flag, a.err))
+          break;
+        const uint32_t e0 = ents[2 * n];
+        const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : (e0 & 0xFFFF0000u);
+        const int r0 = (int)(e0 >> 16) * 64;
+        const int r1 = (int)(e1 >> 16) * 64;
+        uint8_t* kt = smem + L::kKV + st * 2 * L::kTileBytes;
+        uint8_t* vt = kt + L::kTileBytes;
+        mbar_arrive_expect_tx(&bar[kBarKVFull + st], 2 * L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_3d(kt + c * L::kChunkBytes, &tmK, &bar[kBarKVFull + st], c * 64, r0, bh);
+          tma_load_3d(kt + c * L::kChunkBytes + 8192, &tmK, &bar[kBarKVFull + st], c * 64, r1, bh);
+          tma_load_3d(vt + c * L::kChunkBytes, &tmV, &bar[kBarKVFull + st], c * 64, r0, bh);
+          tma_load_3d(vt + c * L::kChunkBytes + 8192, &tmV, &bar[kBarKVFull + st], c * 64, r1, bh);
+        }
+        issued = n + 1;
+      }
+      if (*abort_flag) {  // let copies in flight land before the CTA exits
+        mbar_wait_drain(&bar[kBarQ], 0);
+        for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
+          mbar_wait_drain(&bar[kBarKVFull + (n & 1)], (n >> 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
+      constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, 0, 1);    // P (tmem), V MN-major
+      const uint32_t q_addr = smem_u32(smem + L::kQ);
+      bool ok = mbar_wait(&bar[kBarQ], 0, abort_flag, a.err);
+      tc_fence_after();
+      for (int n = 0; ok && n <= N; ++n) {
+        if (n < N) {
+          const int st = n & 1;
+          if (!mbar_wait(&bar[kBarKVFull + st], (n >> 1) & 1, abort_flag, a.err)) break;
+          // S buffer st holds P(n-2) until PV(n-2) has completed.
+          if (n >= 2 && !mbar_wait(&bar[kBarO], (n - 2) & 1, abort_flag, a.err)) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(smem + L::kKV + st * 2 * L::kTileBytes);
+          const uint32_t s_tmem = tmem + (uint32_t)(st * 128);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (uint32_t)((k >> 2) * L::kChunkBytes + (k & 3) * 32);
+            mma_ss(s_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
+                   smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar[kBarSFull + st]);
+        }
+        if (n >= 1) {
+          const int pn = n - 1;
+          const int pb = pn & 1;
+          if (!mbar_wait(&bar[kBarPFull + pb], (pn >> 1) & 1, abort_flag, a.err)) break;
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(smem + L::kKV + pb * 2 * L::kTileBytes + L::kTileBytes);
+          const uint32_t p_tmem = tmem + (uint32_t)(pb * 128);
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            mma_ts(tmem + 256u, p_tmem + (uint32_t)(k * 8),
+                   smem_desc_sw128(v_addr + (uint32_t)(k * 2048), L::kChunkBytes, 1024), kIdO,
+                   (pn > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[kBarKVEmpty + pb]);
+          mma_commit(&bar[kBarO]);
+        }
+      }
+      mma_commit(&bar[kBarDrain]);
+      mbar_wait_drain(&bar[kBarDrain], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const Dims& d = a.d;
+    const int r = tid;  // query row of the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int qsel = r >> 6;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int n = 0; n < N; ++n) {
+      const int sb = n & 1;
+      ok = mbar_wait(&bar[kBarSFull + sb], (n >> 1) & 1, abort_flag, a.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(tmem + lane_base + (uint32_t)(sb * 128 + 32 * i), s[i]);
+      tmem_wait_ld();
+      const uint32_t e0 = ents[2 * n];
+      const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : 0u;
+      const int lim0 = ((e0 >> qsel) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
+      const int lim1 = ((e1 >> qsel) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int col = 32 * i + c;
+          const bool v = (col < 64) ? (col < lim0) : (col - 64 < lim1);
+          const float x = v ? __uint_as_float(s[i][c]) * a.scale_log2 : -INFINITY;
+          s[i][c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const float base = (m_new == -INFINITY) ? 0.f : m_new;
+      if (n > 0) {
+        // O must hold PV(n-1) before it is rescaled and before PV(n) is issued.
+        ok = mbar_wait(&bar[kBarO], (n - 1) & 1, abort_flag, a.err);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        const float alpha = fast_exp2(m_run - base);
+        if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+          tc_fence_after();
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+          }
+        }
+        l_run *= alpha;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int col = 64 * h2 + 2 * c;
+          const float p0 = fast_exp2(__uint_as_float(s[col >> 5][col & 31]) - base);
+          const float p1 = fast_exp2(__uint_as_float(s[(col + 1) >> 5][(col + 1) & 31]) - base);
+          sum += p0 + p1;
+          pk[c] = pack_bf16(p0, p1);
+        }
+        tmem_st32(tmem + lane_base + (uint32_t)(sb * 128 + 32 * h2), pk);
+      }
+      l_run += sum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar[kBarPFull + sb]);
+      m_run = m_new;
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) {
+      ok = mbar_wait(&bar[kBarO], (N - 1) & 1, abort_flag, a.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int pr = m * kBM + r;  // row in the padded chunk
+      const int f = pr / d.T_pad;
+      const int rr = pr - f * d.T_pad;
+      const bool row_ok = (f < d.Fc) && (rr < d.T_f);
+      const int b = bh / d.H;
+      const int h = bh - b * d.H;
+      const size_t n_tok = (size_t)f * d.T_f + rr;
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      uint16_t* orow = a.out + (((size_t)b * d.Lq + n_tok) * d.H + h) * D;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * i);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (row_ok && a.lse) a.lse[(size_t)bh * d.Lq + n_tok] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- host side --------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3D bf16 map over [d2][d1][d0] (d0 innermost), box (64 columns, box1 rows), 128 B swizzle.
+static bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint32_t box1) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
+                                      const CUtensorMap& mv, cudaStream_t stream) {
+  using L = AttnSmem<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.MT, a.d.B * a.d.H);
+  attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
+                             const void* cache_v, cudaStream_t stream, const char** why) {
+  const Dims& d = a.d;
+  CUtensorMap mq, mk, mv;
+  const uint64_t bh = (uint64_t)d.B * d.H;
+  if (!make_map(&mq, q_rot, d.D, (uint64_t)d.Fc * d.T_pad, bh, 128) ||
+      !make_map(&mk, cache_k, d.D, (uint64_t)a.W * d.T_pad, bh, 64) ||
+      !make_map(&mv, cache_v, d.D, (uint64_t)a.W * d.T_pad, bh, 64)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point or tensor shape)";
+    return cudaErrorInvalidValue;
+  }
+  return d.D == 128 ? launch_attention_d<128>(a, mq, mk, mv, stream)
+                    : launch_attention_d<64>(a, mq, mk, mv, stream);
+}
+
+}  // namespace cva

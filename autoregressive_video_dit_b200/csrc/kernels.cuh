@@ -1,0 +1,77 @@
+// Kernel argument blocks and launchers of libcva (host <-> kernel files).
+#pragma once
+
+#include "cva_internal.cuh"
+
+namespace cva {
+
+// ---- steps 1-3: rotary embedding, cache append, pooling (rope_pool.cu) ----
+enum : int { kTokenMajor = 0, kHeadMajor = 1, kCacheSlots = 2 };
+enum : int { kPoolNone = 0, kPoolChunk = 1, kPoolCache = 2 };
+
+struct StreamJob {
+  const uint16_t* src;  // bf16 input
+  int src_layout;       // kTokenMajor or kHeadMajor
+  uint16_t* dst;        // bf16 output (nullptr: none)
+  int dst_layout;       // kTokenMajor, kHeadMajor or kCacheSlots
+  int rotate;           // apply the rotary embedding
+  float* pool;          // block means (nullptr: none)
+  int pool_layout;      // kPoolChunk or kPoolCache
+};
+
+struct RopePoolArgs {
+  StreamJob job[3];
+  int njobs;
+  RopeTab tab;
+  Dims d;
+  int t0;
+  int W;
+};
+
+struct FramePoolArgs {
+  const float* blk_pool;
+  float* frm_pool;
+  int layout;  // kPoolChunk: [bh][NQB][D] -> [bh][Fc][D]; kPoolCache: [bh][W][nb][D] -> [bh][W][D]
+  Dims d;
+  int t0;
+  int W;
+};
+
+cudaError_t launch_rope_pool(const RopePoolArgs& a, cudaStream_t stream);
+cudaError_t launch_frame_pool(const FramePoolArgs& a, cudaStream_t stream);
+
+// ---- step 4: selection (hsa_select.cu) ----------------------------------
+struct SelectArgs {
+  const float* qpool;      // [B][H][NQB][D]
+  const float* kpool_blk;  // [B][H][W][nb][D]
+  const float* kpool_frm;  // [B][H][W][D]
+  int32_t* frame_idx;      // [B][H][NQB][k_f_stride] or nullptr
+  int32_t* block_idx;      // [B][H][NQB][k_b_max]
+  int32_t* block_cnt;      // [B][H][NQB]
+  Dims d;
+  int W, t_lo, F;          // history frames t_lo .. t_lo+F-1
+  int k_f, k_b, k_f_stride, k_b_max;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+
+// ---- step 5: attention (attn_sm100.cu) -----------------------------------
+struct AttnArgs {
+  const int32_t* block_idx;  // [B][H][NQB][k_b_max] or nullptr (dense)
+  const int32_t* block_cnt;  // [B][H][NQB]
+  int k_b_max;
+  uint16_t* out;             // bf16 [B, Lq, H, D]
+  float* lse;                // [B][H][Lq] or nullptr
+  int* err;                  // device error word
+  Dims d;
+  int W, t0, t_lo, F;
+  int MT;                    // 128-row query tiles per (b, h)
+  float scale_log2;          // log2(e) / sqrt(D)
+};
+constexpr int kAttnMaxEntries = 4096;     // 64-row key units per CTA
+constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
+
+// Builds the tensor maps and launches the attention kernel.
+cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
+                             const void* cache_v, cudaStream_t stream, const char** why);
+
+}  // namespace cva

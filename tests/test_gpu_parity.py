@@ -1,0 +1,517 @@
+"""GPU parity: every step of the CUDA path against the fp64 oracle.
+
+Staged tests feed each kernel the oracle's own (bfloat16-rounded) inputs
+for that step, so a mismatch points at one kernel. End-to-end tests run the
+fused chunk call from raw seeded inputs over a whole sequence of chunks.
+Tolerances: RoPE 1e-2 absolute (or the bf16 rounding bound of the value);
+pooled means 1e-5 relative to the row scale; selection identical except
+where the oracle's boundary gap is below 1e-5 relative; attention max-abs
+2e-2 and mean-abs 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from cva_workload import WORKLOADS, key_centres
+from oracle import hsa as o_hsa
+from oracle import path as o_path
+from oracle import rope as o_rope
+
+from _util import (MAX_ABS, MEAN_ABS, attn_errors, bits_to_f64, f64_to_bits, from_dev, inputs,
+                   lib_budget, oracle_budget, hist_count, rope_tol, sample_rows, selection_mismatch,
+                   shape_of, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["c1", "c1s", "r64", "r128", "r64s"]
+SMALL_SPARSE = ["c1s", "r64", "r128", "r64s"]
+
+
+@pytest.fixture(scope="module")
+def ops():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from autoregressive_video_dit_b200 import ops as _ops
+    _ops.device_status(clear=True)
+    return _ops
+
+
+def _tables(ops, wl, t_begin=0):
+    max_t = t_begin + wl.Fc * max(wl.chunk, wl.chunks) + wl.Fc
+    return ops.DeviceRopeTables(wl.D, max_t, wl.Fh, wl.Fw)
+
+
+def _sub(wl, heads):
+    return wl if heads is None else wl.replace(H=len(heads))
+
+
+def _oracle_run(wl, chunk, heads=None, t_begin=0):
+    """Oracle over the window's chunks; returns per-chunk bf16 values and the
+    final chunk's path outputs (selection, pooled queries) without attention."""
+    H = wl.H if heads is None else len(heads)
+    cache = o_path.FrameCache(wl.B, H, wl.D, wl.T_f, wl.blk, wl.window)
+    cache.t_begin = t_begin
+    centres = key_centres(wl, 0) if wl.keys == "clustered" else None
+    t0_cur = wl.t0_of(chunk) + t_begin
+    lo = max(t_begin, t0_cur + wl.Fc - wl.window)
+    first = (lo - t_begin) // wl.Fc + 1
+    hist = []
+    for c in range(first, chunk):
+        x = inputs(wl, c, 0, heads, centres)
+        q, k, v = (bits_to_f64(x[n]) for n in ("q", "k", "v"))
+        t0 = wl.t0_of(c) + t_begin
+        _, k_rot = o_path.rotate_chunk(q, k, wl.Fh, wl.Fw, wl.Fc, t0, "bf16")
+        cache.append(k_rot, v, t0, wl.Fc)
+        hist.append((t0, k_rot, x["v"]))
+    x = inputs(wl, chunk, 0, heads, centres)
+    q, k, v = (bits_to_f64(x[n]) for n in ("q", "k", "v"))
+    k_f, k_b = oracle_budget(wl, chunk, t_begin)
+    out = o_path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0_cur, k_f=k_f, k_b=k_b,
+                           dense=wl.dense, store="bf16", attend_too=False)
+    out.update(cache=cache, hist=hist, x=x, t0=t0_cur, k_f=k_f, k_b=k_b)
+    return out
+
+
+def _head_major(wl, q_rot_tok):
+    """[B, Lq, H, D] -> [B, H, Fc*T_pad, D] with zero pad rows."""
+    B, Lq, H, D = q_rot_tok.shape
+    out = np.zeros((B, H, wl.Fc, wl.T_pad, D), dtype=q_rot_tok.dtype)
+    x = np.transpose(q_rot_tok, (0, 2, 1, 3)).reshape(B, H, wl.Fc, wl.T_f, D)
+    out[:, :, :, :wl.T_f] = x
+    return out.reshape(B, H, wl.Fc * wl.T_pad, D)
+
+
+def _gpu_cache_from_oracle(ops, wl, run, t_begin=0):
+    """GPU cache holding exactly the oracle's bf16 rotated keys (append without rotation)."""
+    cache = ops.DeviceKVCache(shape_of(wl), wl.window, t_begin)
+    for t0, k_rot, v_bits in run["hist"]:
+        ops.kv_append(to_dev(f64_to_bits(k_rot)), to_dev(v_bits), cache, None, t0)
+    ops.kv_append(to_dev(f64_to_bits(run["k_rot"])), to_dev(run["x"]["v"]), cache, None, run["t0"])
+    return cache
+
+
+# ---- step 1: RoPE ---------------------------------------------------------------
+
+@pytest.mark.parametrize("key", SMALL + ["c2"])
+def test_rope3d_apply(ops, key):
+    import torch
+    wl = WORKLOADS[key]
+    x = inputs(wl, wl.chunk)
+    tabs = _tables(ops, wl)
+    shp = shape_of(wl)
+    for name in ("q", "k"):
+        want = o_rope.rope_chunk(bits_to_f64(x[name]), wl.Fh, wl.Fw, wl.Fc, wl.t0)
+        xd = to_dev(x[name])
+        y0 = torch.empty_like(xd)
+        ops.rope3d_apply(xd, y0, tabs, shp, wl.t0, 0)
+        got = bits_to_f64(from_dev(y0))
+        assert np.all(np.abs(got - want) <= rope_tol(want)), f"{name}: max err {np.abs(got - want).max()}"
+        # exact agreement with the oracle's own bf16 rounding almost everywhere
+        frac_diff = np.mean(got != o_path.round_bf16(want))
+        assert frac_diff < 1e-3
+        y1 = torch.full((wl.B, wl.H, wl.Fc * wl.T_pad, wl.D), float("nan"), dtype=torch.bfloat16,
+                        device="cuda")
+        ops.rope3d_apply(xd, y1, tabs, shp, wl.t0, 1)
+        torch.cuda.synchronize()
+        hm = bits_to_f64(from_dev(y1)).reshape(wl.B, wl.H, wl.Fc, wl.T_pad, wl.D)
+        np.testing.assert_array_equal(hm[:, :, :, :wl.T_f],
+                                      np.transpose(got, (0, 2, 1, 3)).reshape(wl.B, wl.H, wl.Fc, wl.T_f, wl.D))
+        assert np.all(hm[:, :, :, wl.T_f:] == 0)
+
+
+# ---- step 2 (+ K pooling): append ------------------------------------------------------
+
+@pytest.mark.parametrize("key", SMALL)
+def test_kv_append_rotates_copies_and_pools(ops, key):
+    import torch
+    wl = WORKLOADS[key]
+    shp = shape_of(wl)
+    tabs = _tables(ops, wl)
+    cache = ops.DeviceKVCache(shp, wl.window)
+    x = inputs(wl, wl.chunk)
+    ops.kv_append(to_dev(x["k"]), to_dev(x["v"]), cache, tabs, wl.t0)
+    torch.cuda.synchronize()
+    k_want = o_rope.rope_chunk(bits_to_f64(x["k"]), wl.Fh, wl.Fw, wl.Fc, wl.t0)
+    kc = bits_to_f64(from_dev(cache.k))
+    vc = from_dev(cache.v)
+    for f in range(wl.Fc):
+        slot = (wl.t0 + f) % wl.window
+        kf = kc[:, :, slot]                                     # [B,H,T_pad,D]
+        want = np.transpose(k_want[:, f * wl.T_f:(f + 1) * wl.T_f], (0, 2, 1, 3))
+        assert np.all(np.abs(kf[:, :, :wl.T_f] - want) <= rope_tol(want))
+        assert np.all(kf[:, :, wl.T_f:] == 0)
+        np.testing.assert_array_equal(vc[:, :, slot, :wl.T_f],
+                                      np.transpose(x["v"][:, f * wl.T_f:(f + 1) * wl.T_f], (0, 2, 1, 3)))
+        assert np.all(vc[:, :, slot, wl.T_f:] == 0)
+        # pools of the stored keys
+        pb = cache.kpool_blk[:, :, slot].cpu().numpy().astype(np.float64)
+        pf = cache.kpool_frm[:, :, slot].cpu().numpy().astype(np.float64)
+        want_b = o_hsa.block_means(kf[:, :, :wl.T_f], wl.blk)
+        want_f = o_hsa.frame_mean(kf[:, :, :wl.T_f])
+        np.testing.assert_allclose(pb, want_b, rtol=0, atol=2e-6 * max(1.0, np.abs(want_b).max()))
+        np.testing.assert_allclose(pf, want_f, rtol=0, atol=2e-6 * max(1.0, np.abs(want_f).max()))
+
+
+@pytest.mark.parametrize("key", ["r64", "r128"])
+def test_kv_append_without_rotation_is_a_copy(ops, key):
+    import torch
+    wl = WORKLOADS[key]
+    cache = ops.DeviceKVCache(shape_of(wl), wl.window)
+    x = inputs(wl, 2)
+    ops.kv_append(to_dev(x["k"]), to_dev(x["v"]), cache, None, wl.t0_of(2))
+    torch.cuda.synchronize()
+    kc = from_dev(cache.k)
+    for f in range(wl.Fc):
+        slot = (wl.t0_of(2) + f) % wl.window
+        np.testing.assert_array_equal(kc[:, :, slot, :wl.T_f],
+                                      np.transpose(x["k"][:, f * wl.T_f:(f + 1) * wl.T_f], (0, 2, 1, 3)))
+
+
+# ---- step 3: query pooling --------------------------------------------------------------
+
+@pytest.mark.parametrize("key", SMALL + ["c3"])
+def test_hsa_compress(ops, key):
+    import torch
+    wl = WORKLOADS[key]
+    heads = [0, wl.H - 1] if wl.H > 4 else None
+    wl = _sub(wl, heads) if heads else wl
+    x = inputs(WORKLOADS[key], wl.chunk, 0, heads)
+    q_rot, _ = o_path.rotate_chunk(bits_to_f64(x["q"]), bits_to_f64(x["k"]), wl.Fh, wl.Fw, wl.Fc, wl.t0)
+    want_b, want_f = o_path.pool_queries(q_rot, wl.T_f, wl.blk, wl.Fc)
+    qd = to_dev(f64_to_bits(_head_major(wl, q_rot)))
+    pb = torch.empty((wl.B, wl.H, wl.NQB, wl.D), dtype=torch.float32, device="cuda")
+    pf = torch.empty((wl.B, wl.H, wl.Fc, wl.D), dtype=torch.float32, device="cuda")
+    ops.hsa_compress(qd, shape_of(wl), pb, pf)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(pb.cpu().numpy(), want_b, rtol=0, atol=2e-6 * max(1, np.abs(want_b).max()))
+    np.testing.assert_allclose(pf.cpu().numpy(), want_f, rtol=0, atol=2e-6 * max(1, np.abs(want_f).max()))
+
+
+# ---- step 4: selection ------------------------------------------------------------------
+
+def _staged_select(ops, wl, run, t_begin=0):
+    import torch
+    cache = _gpu_cache_from_oracle(ops, wl, run, t_begin)
+    qd = to_dev(f64_to_bits(_head_major(wl, run["q_rot"])))
+    pb = torch.empty((wl.B, wl.H, wl.NQB, wl.D), dtype=torch.float32, device="cuda")
+    ops.hsa_compress(qd, shape_of(wl), pb)
+    k_f, k_b = run["k_f"], run["k_b"]
+    F = len(run["cache"].history(run["t0"], wl.Fc))
+    kfe = min(k_f, F)
+    fi = torch.full((wl.B, wl.H, wl.NQB, max(kfe, 1)), -7, dtype=torch.int32, device="cuda")
+    bi = torch.full((wl.B, wl.H, wl.NQB, max(k_b, 1)), -7, dtype=torch.int32, device="cuda")
+    bc = torch.full((wl.B, wl.H, wl.NQB), -7, dtype=torch.int32, device="cuda")
+    ops.hsa_select(pb, cache, run["t0"], k_f, k_b, fi, bi, bc)
+    torch.cuda.synchronize()
+    return cache, qd, fi.cpu().numpy(), bi.cpu().numpy(), bc.cpu().numpy()
+
+
+@pytest.mark.parametrize("key", SMALL_SPARSE)
+def test_hsa_select_staged(ops, key):
+    wl = WORKLOADS[key]
+    run = _oracle_run(wl, wl.chunk)
+    _, _, fi, bi, bc = _staged_select(ops, wl, run)
+    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    assert bad == 0 and near <= 0.02 * n, (bad, near, n)
+    kfe = run["frames"].shape[-1]
+    ok = (run["gap_f"] >= 1e-5)
+    np.testing.assert_array_equal(fi[..., :kfe][ok], run["frames"][ok])
+
+
+@pytest.mark.parametrize("chunk", [2, 4, 7])
+def test_hsa_select_staged_c3_full_size(ops, chunk):
+    wl = WORKLOADS["c3"].with_chunk(chunk)
+    heads = [0, 5, 11]
+    run = _oracle_run(wl, chunk, heads)
+    k_f, k_b = lib_budget(wl, chunk)
+    assert (k_f, k_b) == (run["k_f"], run["k_b"])
+    _, _, fi, bi, bc = _staged_select(ops, _sub(wl, heads), run)
+    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    assert bad == 0 and near <= 0.02 * n, (bad, near, n)
+
+
+# ---- step 5: attention ------------------------------------------------------------------
+
+def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0):
+    import torch
+    cache = _gpu_cache_from_oracle(ops, wl, run, t_begin)
+    qd = to_dev(f64_to_bits(_head_major(wl, run["q_rot"])))
+    out = torch.full((wl.B, wl.Lq, wl.H, wl.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((wl.B, wl.H, wl.Lq), float("nan"), dtype=torch.float32, device="cuda")
+    if blocks is None:
+        ops.blocksparse_attn_fwd(qd, cache, run["t0"], None, None, 0, out, lse)
+    else:
+        kb = blocks.shape[-1]
+        # at least one element: an empty tensor has a NULL data pointer, which means "dense"
+        padded = np.zeros(blocks.shape[:-1] + (max(kb, 1),), dtype=np.int32)
+        padded[..., :kb] = blocks
+        bi = torch.from_numpy(padded).cuda()
+        bc = torch.full(blocks.shape[:-1], kb, dtype=torch.int32, device="cuda")
+        ops.blocksparse_attn_fwd(qd, cache, run["t0"], bi, bc, kb, out, lse)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o_want, l_want = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, blocks, rows)
+    got = bits_to_f64(from_dev(out))
+    gl = lse.cpu().numpy().astype(np.float64)
+    sel = np.arange(wl.Lq) if rows is None else rows
+    mx, mean, rel = attn_errors(got[:, sel], o_want[:, sel])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+    np.testing.assert_allclose(gl[:, :, sel], l_want[:, :, sel], rtol=0, atol=2e-3)
+    return mx, mean, rel
+
+
+@pytest.mark.parametrize("key", SMALL)
+def test_attention_staged(ops, key):
+    wl = WORKLOADS[key]
+    run = _oracle_run(wl, wl.chunk)
+    _check_attention(ops, wl, run, run["blocks"])
+
+
+@pytest.mark.parametrize("key", SMALL_SPARSE)
+def test_attention_staged_dense_call(ops, key):
+    # block_idx == NULL: every history block
+    wl = WORKLOADS[key]
+    run = _oracle_run(wl, wl.chunk)
+    _check_attention(ops, wl, run, None)
+
+
+def test_attention_staged_c2_full_size_sampled(ops):
+    wl = WORKLOADS["c2"]
+    heads = [3, 10]
+    run = _oracle_run(wl, wl.chunk, heads)
+    rows = sample_rows(wl, 2, np.random.default_rng(1))
+    _check_attention(ops, _sub(wl, heads), run, None, rows)
+
+
+def test_attention_staged_c4_full_size_sampled(ops):
+    wl = WORKLOADS["c4"]
+    heads = [7]
+    run = _oracle_run(wl, wl.chunk, heads)
+    rows = sample_rows(wl, 2, np.random.default_rng(2))
+    _check_attention(ops, _sub(wl, heads), run, run["blocks"], rows)
+
+
+# ---- whole path --------------------------------------------------------------------------
+
+def _gpu_stream(ops, wl, upto, t_begin=0, heads=None, record=()):
+    """Run the fused chunk call for chunks 1..upto; returns outputs of `record` chunks."""
+    import torch
+    wlh = _sub(wl, heads)
+    shp = shape_of(wlh)
+    tabs = _tables(ops, wl, t_begin)
+    cache = ops.DeviceKVCache(shp, wl.window, t_begin)
+    centres = key_centres(wl, 0) if wl.keys == "clustered" else None
+    res = {}
+    for c in range(1, upto + 1):
+        x = inputs(wl, c, 0, heads, centres)
+        t0 = wl.t0_of(c) + t_begin
+        k_f, k_b = lib_budget(wl, c, t_begin)
+        if wl.dense:
+            k_f, k_b = -1, 0
+        ws = torch.empty(ops.chunk_workspace_bytes(shp, k_f, k_b), dtype=torch.uint8, device="cuda")
+        out = torch.empty((wlh.B, wlh.Lq, wlh.H, wlh.D), dtype=torch.bfloat16, device="cuda")
+        ops.chunk_attention(to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]), cache, tabs, t0, k_f, k_b, ws, out)
+        if c in record or c == upto:
+            torch.cuda.synchronize()
+            res[c] = (from_dev(out), ws, k_f, k_b)
+    assert ops.device_status() == 0
+    return res, cache
+
+
+def _e2e_compare(wl, run, gpu_out, blocks_ok=None, rows=None):
+    """Output of the fused call vs the oracle; query blocks where the
+    selection differed (near ties) are excluded."""
+    o_want, _ = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, run["blocks"], rows)
+    got = bits_to_f64(gpu_out)
+    sel = np.arange(wl.Lq) if rows is None else rows
+    g = got[:, sel]
+    w = o_want[:, sel]
+    if blocks_ok is not None:
+        qb = (sel // wl.T_f) * wl.nb + (sel % wl.T_f) // wl.blk
+        mask = blocks_ok[:, :, qb]                          # [B, H, rows]
+        mask = np.transpose(mask, (0, 2, 1))[..., None]     # [B, rows, H, 1]
+        g = np.where(mask, g, 0.0)
+        w = np.where(mask, w, 0.0)
+    return attn_errors(g, w)
+
+
+def _selection_ok_mask(run, gpu_blocks):
+    if run["blocks"] is None:
+        return None
+    kb = run["blocks"].shape[-1]
+    return np.all(gpu_blocks[..., :kb] == run["blocks"], axis=-1)
+
+
+def _ws_blocks(ops, wl, ws, k_f, k_b):
+    """Block lists the fused call wrote into its workspace (layout of cva_chunk_workspace_bytes)."""
+    d = wl
+    bhq = d.B * d.H * d.NQB
+    r256 = lambda x: (x + 255) // 256 * 256
+    off = r256(d.B * d.H * d.Fc * d.T_pad * d.D * 2) + r256(bhq * d.D * 4) + r256(bhq * max(k_f, 0) * 4)
+    raw = ws[off:off + bhq * k_b * 4].cpu().numpy().view(np.int32)
+    return raw.reshape(d.B, d.H, d.NQB, k_b)
+
+
+@pytest.mark.parametrize("key", SMALL)
+def test_chunk_attention_end_to_end(ops, key):
+    wl = WORKLOADS[key]
+    res, _ = _gpu_stream(ops, wl, wl.chunk)
+    out, ws, k_f, k_b = res[wl.chunk]
+    run = _oracle_run(wl, wl.chunk)
+    ok = None
+    if not wl.dense and k_b > 0:
+        gb = _ws_blocks(ops, wl, ws, k_f, k_b)
+        ok = _selection_ok_mask(run, gb)
+        assert ok.mean() >= 0.98, ok.mean()
+    mx, mean, rel = _e2e_compare(wl, run, out, ok)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+def test_chunk_attention_global_time_shift(ops):
+    # the same stream started at global frame 100: identical outputs up to
+    # rounding of the rotated values, and parity with the oracle
+    wl = WORKLOADS["c1s"]
+    a, _ = _gpu_stream(ops, wl, wl.chunk, 0)
+    b, _ = _gpu_stream(ops, wl, wl.chunk, 100)
+    run = _oracle_run(wl, wl.chunk, None, 100)
+    mx, mean, _ = _e2e_compare(wl, run, b[wl.chunk][0])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS
+    d = np.abs(bits_to_f64(a[wl.chunk][0]) - bits_to_f64(b[wl.chunk][0]))
+    assert d.max() <= 2 * MAX_ABS
+
+
+def test_chunk_attention_rolling_window_wrap(ops):
+    # window of 8 frames over 7 chunks of 3: slots wrap twice
+    wl = WORKLOADS["r64s"].with_chunk(7)
+    res, cache = _gpu_stream(ops, wl, 7)
+    out, ws, k_f, k_b = res[7]
+    run = _oracle_run(wl, 7)
+    assert cache.history_frames(run["t0"]) == (13, 5)
+    gb = _ws_blocks(ops, wl, ws, k_f, k_b)
+    ok = _selection_ok_mask(run, gb)
+    mx, mean, _ = _e2e_compare(wl, run, out, ok)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS
+
+
+def test_chunk_attention_first_chunk_has_no_history(ops):
+    wl = WORKLOADS["r128"].with_chunk(1)
+    res, _ = _gpu_stream(ops, wl, 1)
+    run = _oracle_run(wl, 1)
+    mx, mean, _ = _e2e_compare(wl, run, res[1][0])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS
+
+
+def test_c2_dense_end_to_end_sampled(ops):
+    wl = WORKLOADS["c2"]
+    res, _ = _gpu_stream(ops, wl, wl.chunk)
+    heads = [0, 11]
+    run = _oracle_run(wl, wl.chunk, heads)
+    rows = sample_rows(wl, 1, np.random.default_rng(3))
+    out = res[wl.chunk][0][:, :, heads]
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out, None, rows)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+@pytest.mark.parametrize("chunk", [2, 7])
+def test_c3_hsa_end_to_end_sampled(ops, chunk):
+    wl = WORKLOADS["c3"].with_chunk(chunk)
+    res, _ = _gpu_stream(ops, wl, chunk)
+    out, ws, k_f, k_b = res[chunk]
+    heads = [1, 6]
+    run = _oracle_run(wl, chunk, heads)
+    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
+    ok = _selection_ok_mask(run, gb)
+    assert ok.mean() >= 0.98, ok.mean()
+    rows = sample_rows(wl, 1, np.random.default_rng(4))
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+def test_c4_end_to_end_sampled(ops):
+    wl = WORKLOADS["c4"]
+    heads = [0, 21, 39]
+    res, _ = _gpu_stream(ops, wl, wl.chunk)
+    out, ws, k_f, k_b = res[wl.chunk]
+    run = _oracle_run(wl, wl.chunk, heads)
+    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
+    ok = _selection_ok_mask(run, gb)
+    assert ok.mean() >= 0.98, ok.mean()
+    rows = sample_rows(wl, 1, np.random.default_rng(5), blocks=range(0, wl.NQB, 3))
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+def test_c5_streaming_window_sampled(ops):
+    # 1.3B shape, rolling window of 60 frames: check chunk 21 (window full)
+    # on two heads; the GPU runs every head of every chunk.
+    wl = WORKLOADS["c5"].with_chunk(21)
+    heads = [2, 9]
+    res, cache = _gpu_stream(ops, wl, 21)
+    out, ws, k_f, k_b = res[21]
+    assert (k_f, k_b) == (20, 285)
+    assert cache.history_frames(wl.t0_of(21)) == (3, 57)
+    run = _oracle_run(wl, 21, heads)
+    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
+    ok = _selection_ok_mask(run, gb)
+    assert ok.mean() >= 0.98, ok.mean()
+    rows = sample_rows(wl, 1, np.random.default_rng(6), blocks=range(0, wl.NQB, 4))
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+# ---- edge cases and errors ------------------------------------------------------------------
+
+def test_zero_blocks_attends_current_chunk_only(ops):
+    wl = WORKLOADS["r64"]
+    run = _oracle_run(wl, wl.chunk)
+    empty = np.zeros(run["blocks"].shape[:-1] + (0,), dtype=np.int64)
+    _check_attention(ops, wl, run, empty)
+
+
+def test_single_block_budget(ops):
+    wl = WORKLOADS["r128"]
+    run = _oracle_run(wl, wl.chunk)
+    sel = o_path.select_chunk(run["qbar_blk"], run["cache"], run["cache"].history(run["t0"], wl.Fc), 1, 1)
+    _check_attention(ops, wl, run, sel[1])
+
+
+def test_bad_block_index_is_latched_not_read(ops):
+    import torch
+    wl = WORKLOADS["r64"]
+    run = _oracle_run(wl, wl.chunk)
+    cache = _gpu_cache_from_oracle(ops, wl, run)
+    qd = to_dev(f64_to_bits(_head_major(wl, run["q_rot"])))
+    blocks = run["blocks"].astype(np.int32).copy()
+    blocks[0, 0, 0, 0] = 10 ** 6          # far outside the cache window
+    bi = torch.from_numpy(blocks).cuda()
+    bc = torch.full(blocks.shape[:-1], blocks.shape[-1], dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    ops.blocksparse_attn_fwd(qd, cache, run["t0"], bi, bc, blocks.shape[-1], out)
+    torch.cuda.synchronize()
+    assert ops.device_status(clear=True) == ops.DEV_BAD_INDEX
+    assert ops.device_status() == 0
+
+
+def test_host_errors(ops):
+    import torch
+    wl = WORKLOADS["r64"]
+    shp = shape_of(wl)
+    tabs = ops.DeviceRopeTables(wl.D, 8, wl.Fh, wl.Fw)
+    cache = ops.DeviceKVCache(shp, wl.window)
+    q = torch.zeros((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ops.CvaError) as e:
+        ops.chunk_attention(q, q, q, cache, tabs, 9, -1, 0, ws, out)   # t0 + Fc > max_t
+    assert e.value.code == ops.CVA_ERANGE
+    tabs2 = ops.DeviceRopeTables(wl.D, 64, wl.Fh, wl.Fw)
+    with pytest.raises(ops.CvaError) as e:
+        ops.chunk_attention(q, q, q, cache, tabs2, 6, -1, 0, ws, out)  # workspace too small
+    assert e.value.code == ops.CVA_ENOMEM
+    ws = torch.empty(ops.chunk_workspace_bytes(shp, 4, 9), dtype=torch.uint8, device="cuda")
+    with pytest.raises(ops.CvaError) as e:
+        ops.chunk_attention(q, q, q, cache, tabs2, 6, 4, 9, ws, out)   # k_b > k_f * nb = 8
+    assert e.value.code == ops.CVA_ERANGE
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
