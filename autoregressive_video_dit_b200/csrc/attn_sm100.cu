@@ -14,13 +14,16 @@
 // Roles (192 threads):
 //   warp 4 (one lane): TMA producer. Q once; then K and V of each key tile,
 //     gathered by block index with one 64-row box per unit and 64-column
-//     chunk, 128-byte swizzle, into a 2-stage ring. No multicast.
-//   warp 5 (one lane): tcgen05.mma issuer. S(n) = Q K(n)^T into one of two
-//     128-column fp32 TMEM buffers; O += P(n) V(n) with P read from TMEM
-//     (bf16, aliased onto the S buffer) and O in TMEM.
+//     chunk, 128-byte swizzle, into a K slot and a V slot (K(n+1) lands
+//     while the softmax of tile n runs). No multicast.
+//   warp 5 (one lane): tcgen05.mma issuer. S(n) = Q K(n)^T into 128 fp32
+//     TMEM columns; O += P(n) V(n) with P read from TMEM (bf16, aliased onto
+//     the S columns) and O in TMEM.
 //   warps 0-3: softmax; thread i owns query row i (TMEM lane i): masks,
-//     online max/sum in fp32 (exp2 domain), rescales O in TMEM when the
-//     running max moves, writes P, and finally normalises O into bf16.
+//     online max/sum in fp32 (exp2 domain, packed f32x2 arithmetic), O is
+//     rescaled in TMEM only when the row maximum grows by more than 2^8,
+//     writes P, and finally normalises O into bf16.
+// Two CTAs run per SM, so one CTA's softmax overlaps the other's MMAs.
 // Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
 // roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait and the tensor memory is released.
@@ -34,17 +37,20 @@ namespace cva {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kAttnThreads = 192;
-constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;   // S (128 fp32 columns, P aliased onto it) + O (128)
+constexpr uint32_t kOCol = 128;
 
+// Two CTAs share an SM (each ~108 KB of smem, 256 TMEM columns): one CTA's
+// softmax overlaps the other's tensor-core work.
 template <int D>
 struct AttnSmem {
   static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B: one 64-column chunk
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // a Q, K or V tile
   static constexpr int kQ = 0;
-  static constexpr int kKV = kQ + kTileBytes;  // stage s: K at kKV + 2*s*tile, V after it
-  static constexpr int kEnt = kKV + kStages * 2 * kTileBytes;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + kTileBytes;
+  static constexpr int kEnt = kV + kTileBytes;
   static constexpr int kBm = kEnt + kAttnMaxEntries * 4;
   static constexpr int kScan = kBm + 2 * kAttnMaxBitmapWords * 4;
   static constexpr int kBar = kScan + kAttnMaxBitmapWords * 4;
@@ -53,14 +59,47 @@ struct AttnSmem {
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
 };
 
-// Barrier slots.
-enum : int { kBarQ = 0, kBarKVFull = 1, kBarKVEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarO = 9,
-             kBarDrain = 10 };
+// Barrier slots (each completes once per key tile, except Q and drain).
+enum : int { kBarQ = 0, kBarKFull = 1, kBarVFull = 2, kBarKEmpty = 3, kBarVEmpty = 4, kBarSFull = 5,
+             kBarPFull = 6, kBarO = 7, kBarDrain = 8 };
+
+// Above this growth of the row maximum (log2 units) O is rescaled; below
+// it the stale maximum is kept, so P <= 2^8.
+constexpr float kRescaleThreshold = 8.0f;
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (a * b + c) on a pair of floats in one packed instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // A wait with its own limit that ignores the abort flag (used while draining).
@@ -184,7 +223,7 @@ __device__ int build_units(const AttnArgs& a, int m, int bh, uint32_t* ents, uin
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using L = AttnSmem<D>;
@@ -204,12 +243,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bar[kBarQ], 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar[kBarKVFull + s], 1);
-      mbar_init(&bar[kBarKVEmpty + s], 1);
-      mbar_init(&bar[kBarSFull + s], 1);
-      mbar_init(&bar[kBarPFull + s], 128);
-    }
+    mbar_init(&bar[kBarKFull], 1);
+    mbar_init(&bar[kBarVFull], 1);
+    mbar_init(&bar[kBarKEmpty], 1);
+    mbar_init(&bar[kBarVEmpty], 1);
+    mbar_init(&bar[kBarSFull], 1);
+    mbar_init(&bar[kBarPFull], 128);
     mbar_init(&bar[kBarO], 1);
     mbar_init(&bar[kBarDrain], 1);
     *abort_flag = 0;
@@ -229,6 +268,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
+    // K(n) goes into the K slot once S(n-1) has consumed it; V(n) into the V
+    // slot once PV(n-1) has.
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -236,30 +277,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
         tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int n = 0; n < N; ++n) {
-        const int st = n & 1;
-        if (n >= 2 && !mbar_wait(&bar[kBarKVEmpty + st], ((n - 2) >> 1) & 1, abort_flag, a.err))
-          break;
         const uint32_t e0 = ents[2 * n];
         const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : (e0 & 0xFFFF0000u);
         const int r0 = (int)(e0 >> 16) * 64;
         const int r1 = (int)(e1 >> 16) * 64;
-        uint8_t* kt = smem + L::kKV + st * 2 * L::kTileBytes;
-        uint8_t* vt = kt + L::kTileBytes;
-        mbar_arrive_expect_tx(&bar[kBarKVFull + st], 2 * L::kTileBytes);
+        if (n >= 1 && !mbar_wait(&bar[kBarKEmpty], (n - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(&bar[kBarKFull], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(kt + c * L::kChunkBytes, &tmK, &bar[kBarKVFull + st], c * 64, r0, bh);
-          tma_load_3d(kt + c * L::kChunkBytes + 8192, &tmK, &bar[kBarKVFull + st], c * 64, r1, bh);
-          tma_load_3d(vt + c * L::kChunkBytes, &tmV, &bar[kBarKVFull + st], c * 64, r0, bh);
-          tma_load_3d(vt + c * L::kChunkBytes + 8192, &tmV, &bar[kBarKVFull + st], c * 64, r1, bh);
+          tma_load_3d(smem + L::kK + c * L::kChunkBytes, &tmK, &bar[kBarKFull], c * 64, r0, bh);
+          tma_load_3d(smem + L::kK + c * L::kChunkBytes + 8192, &tmK, &bar[kBarKFull], c * 64, r1, bh);
         }
-        issued = n + 1;
+        k_issued = n + 1;
+        if (n >= 1 && !mbar_wait(&bar[kBarVEmpty], (n - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(&bar[kBarVFull], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_3d(smem + L::kV + c * L::kChunkBytes, &tmV, &bar[kBarVFull], c * 64, r0, bh);
+          tma_load_3d(smem + L::kV + c * L::kChunkBytes + 8192, &tmV, &bar[kBarVFull], c * 64, r1, bh);
+        }
+        v_issued = n + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
         mbar_wait_drain(&bar[kBarQ], 0);
-        for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
-          mbar_wait_drain(&bar[kBarKVFull + (n & 1)], (n >> 1) & 1);
+        if (k_issued) mbar_wait_drain(&bar[kBarKFull], (k_issued - 1) & 1);
+        if (v_issued) mbar_wait_drain(&bar[kBarVFull], (v_issued - 1) & 1);
       }
     }
   } else if (warp == 5) {
@@ -268,41 +310,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, 0, 1);    // P (tmem), V MN-major
       const uint32_t q_addr = smem_u32(smem + L::kQ);
+      const uint32_t k_addr = smem_u32(smem + L::kK);
+      const uint32_t v_addr = smem_u32(smem + L::kV);
       bool ok = mbar_wait(&bar[kBarQ], 0, abort_flag, a.err);
-      tc_fence_after();
-      for (int n = 0; ok && n <= N; ++n) {
-        if (n < N) {
-          const int st = n & 1;
-          if (!mbar_wait(&bar[kBarKVFull + st], (n >> 1) & 1, abort_flag, a.err)) break;
-          // S buffer st holds P(n-2) until PV(n-2) has completed.
-          if (n >= 2 && !mbar_wait(&bar[kBarO], (n - 2) & 1, abort_flag, a.err)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + L::kKV + st * 2 * L::kTileBytes);
-          const uint32_t s_tmem = tmem + (uint32_t)(st * 128);
+      for (int n = 0; ok && n < N; ++n) {
+        const uint32_t par = n & 1;
+        if (!mbar_wait(&bar[kBarKFull], par, abort_flag, a.err)) break;
+        // P(n-1) lives in the S columns and O must be final before rescaling:
+        // PV(n-1) has to complete before S(n) is issued.
+        if (n >= 1 && !mbar_wait(&bar[kBarO], (n - 1) & 1, abort_flag, a.err)) break;
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (uint32_t)((k >> 2) * L::kChunkBytes + (k & 3) * 32);
-            mma_ss(s_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
-                   smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar[kBarSFull + st]);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (uint32_t)((k >> 2) * L::kChunkBytes + (k & 3) * 32);
+          mma_ss(tmem, smem_desc_sw128(q_addr + off, 16, 1024),
+                 smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
         }
-        if (n >= 1) {
-          const int pn = n - 1;
-          const int pb = pn & 1;
-          if (!mbar_wait(&bar[kBarPFull + pb], (pn >> 1) & 1, abort_flag, a.err)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + L::kKV + pb * 2 * L::kTileBytes + L::kTileBytes);
-          const uint32_t p_tmem = tmem + (uint32_t)(pb * 128);
+        mma_commit(&bar[kBarSFull]);
+        mma_commit(&bar[kBarKEmpty]);
+        if (!mbar_wait(&bar[kBarPFull], par, abort_flag, a.err)) break;
+        if (!mbar_wait(&bar[kBarVFull], par, abort_flag, a.err)) break;
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            mma_ts(tmem + 256u, p_tmem + (uint32_t)(k * 8),
-                   smem_desc_sw128(v_addr + (uint32_t)(k * 2048), L::kChunkBytes, 1024), kIdO,
-                   (pn > 0 || k > 0) ? 1u : 0u);
-          }
-          mma_commit(&bar[kBarKVEmpty + pb]);
-          mma_commit(&bar[kBarO]);
+        for (int k = 0; k < kBN / 16; ++k) {
+          mma_ts(tmem + kOCol, tmem + (uint32_t)(k * 8),
+                 smem_desc_sw128(v_addr + (uint32_t)(k * 2048), L::kChunkBytes, 1024), kIdO,
+                 (n > 0 || k > 0) ? 1u : 0u);
         }
+        mma_commit(&bar[kBarO]);
+        mma_commit(&bar[kBarVEmpty]);
       }
       mma_commit(&bar[kBarDrain]);
       mbar_wait_drain(&bar[kBarDrain], 0);
@@ -311,78 +347,103 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ softmax
     const Dims& d = a.d;
     const int r = tid;  // query row of the tile = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int qsel = r >> 6;
-    float m_run = -INFINITY;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int qsel = r >> 6;   // warp-uniform
+    const float sc = a.scale_log2;
+    float m_used = -INFINITY;  // running maximum in scaled log2 units (possibly stale by < 8)
     float l_run = 0.f;
     bool ok = true;
     for (int n = 0; n < N; ++n) {
-      const int sb = n & 1;
-      ok = mbar_wait(&bar[kBarSFull + sb], (n >> 1) & 1, abort_flag, a.err);
+      ok = mbar_wait(&bar[kBarSFull], n & 1, abort_flag, a.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld32(tmem + lane_base + (uint32_t)(sb * 128 + 32 * i), s[i]);
-      tmem_wait_ld();
       const uint32_t e0 = ents[2 * n];
       const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : 0u;
       const int lim0 = ((e0 >> qsel) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
       const int lim1 = ((e1 >> qsel) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
+      const bool full = (lim0 == 64) && (lim1 == 64);   // warp-uniform
+
+      // pass 1: row maximum of the raw scores over the valid columns
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(trow + (uint32_t)(64 * h), s0);
+        tmem_ld32(trow + (uint32_t)(64 * h + 32), s1);
+        tmem_wait_ld();
+        const int lim = h == 0 ? lim0 : lim1;
+        if (full) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = 32 * i + c;
-          const bool v = (col < 64) ? (col < lim0) : (col - 64 < lim1);
-          const float x = v ? __uint_as_float(s[i][c]) * a.scale_log2 : -INFINITY;
-          s[i][c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < 32; c += 2) {
+            mx = max3f(mx, __uint_as_float(s0[c]), __uint_as_float(s0[c + 1]));
+            mx = max3f(mx, __uint_as_float(s1[c]), __uint_as_float(s1[c + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < lim) mx = fmaxf(mx, __uint_as_float(s0[c]));
+            if (c + 32 < lim) mx = fmaxf(mx, __uint_as_float(s1[c]));
+          }
         }
       }
-      const float m_new = fmaxf(m_run, mx);
-      const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      if (n > 0) {
-        // O must hold PV(n-1) before it is rescaled and before PV(n) is issued.
-        ok = mbar_wait(&bar[kBarO], (n - 1) & 1, abort_flag, a.err);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) break;
-        const float alpha = fast_exp2(m_run - base);
-        if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
-          tc_fence_after();
+      const float mt = mx * sc;  // -inf when nothing is valid
+      const bool need = mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt > -INFINITY);
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        const float m_new = need ? mt : m_used;
+        const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
+        if (n > 0) {
+          // O holds PV(0..n-1) (complete: S(n) was issued after PV(n-1)).
 #pragma unroll
           for (int i = 0; i < D / 32; ++i) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+            tmem_ld32(trow + kOCol + (uint32_t)(32 * i), o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+            tmem_st32(trow + kOCol + (uint32_t)(32 * i), o);
           }
         }
         l_run *= alpha;
+        m_used = m_new;
       }
-      float sum = 0.f;
+      const float base = (m_used == -INFINITY) ? 0.f : m_used;
+      const float2 sc2 = make_float2(sc, sc);
+      const float2 nb2 = make_float2(-base, -base);
+
+      // pass 2: P = exp2(s * scale - base), row sum, bf16 P into the S columns
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(trow + (uint32_t)(64 * h), s0);
+        tmem_ld32(trow + (uint32_t)(64 * h + 32), s1);
+        tmem_wait_ld();
+        const int lim = h == 0 ? lim0 : lim1;
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = 64 * h2 + 2 * c;
-          const float p0 = fast_exp2(__uint_as_float(s[col >> 5][col & 31]) - base);
-          const float p1 = fast_exp2(__uint_as_float(s[(col + 1) >> 5][(col + 1) & 31]) - base);
-          sum += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
+        for (int c = 0; c < 32; c += 2) {
+          float2 x0 = ffma2(make_float2(__uint_as_float(s0[c]), __uint_as_float(s0[c + 1])), sc2, nb2);
+          float2 x1 = ffma2(make_float2(__uint_as_float(s1[c]), __uint_as_float(s1[c + 1])), sc2, nb2);
+          if (!full) {
+            if (c >= lim) x0.x = -INFINITY;
+            if (c + 1 >= lim) x0.y = -INFINITY;
+            if (c + 32 >= lim) x1.x = -INFINITY;
+            if (c + 33 >= lim) x1.y = -INFINITY;
+          }
+          const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
+          const float2 p1 = make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
+          acc0 = fadd2(acc0, p0);
+          acc1 = fadd2(acc1, p1);
+          pk[c >> 1] = cvt_bf16x2(p0.x, p0.y);
+          pk[16 + (c >> 1)] = cvt_bf16x2(p1.x, p1.y);
         }
-        tmem_st32(tmem + lane_base + (uint32_t)(sb * 128 + 32 * h2), pk);
+        tmem_st32(trow + (uint32_t)(32 * h), pk);
       }
-      l_run += sum;
+      l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[kBarPFull + sb]);
-      m_run = m_new;
+      mbar_arrive(&bar[kBarPFull]);
     }
     // ------------------------------------------------------------ epilogue
     if (ok) {
@@ -403,20 +464,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + 256u + (uint32_t)(32 * i), o);
+        tmem_ld32(trow + kOCol + (uint32_t)(32 * i), o);
         tmem_wait_ld();
         if (row_ok) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            pk[c] = pack_bf16(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+            pk[c] = cvt_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * i);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (row_ok && a.lse) a.lse[(size_t)bh * d.Lq + n_tok] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (row_ok && a.lse)
+        a.lse[(size_t)bh * d.Lq + n_tok] = (m_used + log2f(l_run)) * 0.69314718055994531f;
     }
   }
 
@@ -463,6 +525,8 @@ static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, 
   using L = AttnSmem<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::kAlloc);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(a.MT, a.d.B * a.d.H);
   attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
