@@ -83,6 +83,7 @@ _SIGS = {
                                       c_int32, c_int32, c_int32, c_void_p, c_size_t, c_void_p,
                                       c_void_p, c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
+    "cva_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
     "cva_kv_cache_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
     "cva_kv_cache_init": (c_int32, [P(KVCache), c_void_p, c_size_t, P(Shape), c_int32, c_int32]),
     "cva_cag_budget": (c_int32, [P(CagCfg), c_int32, c_int32, c_int32, P(c_int32), P(c_int32)]),
@@ -197,6 +198,11 @@ def set_stage_events(events) -> None:
         return
     arr = (c_void_p * 4)(*[int(e.cuda_event) for e in events])
     check(lib.cva_set_stage_events(arr, len(events)))
+
+
+def exp2_poly_eval(x, y, stream=None) -> None:
+    """Diagnostic: the softmax's polynomial exp2 on a float32 device tensor."""
+    check(lib.cva_exp2_poly_eval(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
 def device_status(clear: bool = True) -> int:

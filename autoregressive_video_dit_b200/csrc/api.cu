@@ -197,6 +197,14 @@ int cva_set_stage_events(void* const* events, int32_t n) {
   return CVA_OK;
 }
 
+int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream) {
+  if (n < 0) return fail(CVA_EINVAL, "n < 0");
+  if (n == 0) return CVA_OK;
+  if (!x || !y) return fail(CVA_EINVAL, "x or y is NULL");
+  cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "exp2_poly_eval launch");
+}
+
 int cva_rope_axis_pairs(int32_t head_dim, int32_t* p_t, int32_t* p_h, int32_t* p_w) {
   if (!p_t || !p_h || !p_w) return fail(CVA_EINVAL, "NULL output");
   if (head_dim < 6 || head_dim % 2) return fail(CVA_EINVAL, "head_dim must be even and >= 6");

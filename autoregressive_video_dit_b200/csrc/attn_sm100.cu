@@ -4,26 +4,30 @@
 // picked frame-block pairs, here together with every token of the current
 // chunk; its cost is independent of how long the history is.
 //
-// One CTA computes a 128-row query tile of one (batch, head). Its key set
-// is a list of 64-row key units in smem: the union of the picked history
-// blocks of the tile's query blocks (two 64-token query blocks share a tile
-// when blk = 64; a unit carries a 2-bit mask of the query blocks that
-// picked it) followed by the current chunk's blocks. Pairs of units form
-// 128-key tiles.
+// A CTA owns one SM and works on two 128-row query tiles of one (batch,
+// head) at once, in two independent lanes (A and B). Each lane has its own
+// key list, its own Q, K and V tiles in shared memory and its own S and O
+// accumulators in tensor memory (4 x 128 columns). A key list is a list of
+// 64-row key units: the union of the picked history blocks of the lane's
+// query blocks (two 64-token query blocks share a tile when blk = 64; a unit
+// carries a 2-bit mask of the query blocks that picked it), followed by the
+// current chunk's blocks. Pairs of units form 128-key tiles.
 //
-// Roles (192 threads):
-//   warp 4 (one lane): TMA producer. Q once; then K and V of each key tile,
-//     gathered by block index with one 64-row box per unit and 64-column
-//     chunk, 128-byte swizzle, into a K slot and a V slot (K(n+1) lands
-//     while the softmax of tile n runs). No multicast.
-//   warp 5 (one lane): tcgen05.mma issuer. S(n) = Q K(n)^T into 128 fp32
-//     TMEM columns; O += P(n) V(n) with P read from TMEM (bf16, aliased onto
-//     the S columns) and O in TMEM.
-//   warps 0-3: softmax; thread i owns query row i (TMEM lane i): masks,
-//     online max/sum in fp32 (exp2 domain, packed f32x2 arithmetic), O is
-//     rescaled in TMEM only when the row maximum grows by more than 2^8,
-//     writes P, and finally normalises O into bf16.
-// Two CTAs run per SM, so one CTA's softmax overlaps the other's MMAs.
+// Roles (384 threads):
+//   warps 0-3 / 4-7: softmax of lane A / B; thread i owns query row i
+//     (TMEM lane i). One tensor-memory load brings the 128 scores of a tile
+//     into registers; masks, row maximum (3-input max), exp2 on the MUFU in
+//     fp32 with packed f32x2 arithmetic, bf16 P written back over the S
+//     columns. O is rescaled in tensor memory only when the row maximum grows
+//     by more than 2^8. Finally O is normalised into bf16.
+//   warp 8 (one lane): TMA producer. Q once per lane; then per key tile K
+//     into the lane's K slot (free once S of the previous tile completed) and
+//     V into its V slot (free once PV completed), gathered by block index
+//     with one 64-row box per unit and 64-column chunk, 128-byte swizzle.
+//     No multicast.
+//   warp 9 (one lane): tcgen05.mma issuer, interleaving the lanes:
+//     PV_A(n), S_A(n+1), PV_B(n), S_B(n+1), ... so that one lane's MMAs run
+//     while the other lane's softmax does.
 // Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
 // roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait and the tensor memory is released.
@@ -36,32 +40,36 @@ namespace cva {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kAttnThreads = 192;
-constexpr uint32_t kTmemCols = 256;   // S (128 fp32 columns, P aliased onto it) + O (128)
+constexpr int kLanes = 2;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+// 12 warps: registers are granted per group of four warps, so warps 10 and
+// 11 cost nothing extra; they only join the final barrier.
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kTmemCols = 512;   // lane x: S at 256x (P aliased onto it), O at 256x + 128
 constexpr uint32_t kOCol = 128;
 
-// Two CTAs share an SM (each ~108 KB of smem, 256 TMEM columns): one CTA's
-// softmax overlaps the other's tensor-core work.
 template <int D>
 struct AttnSmem {
   static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B: one 64-column chunk
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // a Q, K or V tile
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kTileBytes;
-  static constexpr int kEnt = kV + kTileBytes;
-  static constexpr int kBm = kEnt + kAttnMaxEntries * 4;
+  static constexpr int kQ = 0;                              // lane x at + x * tile
+  static constexpr int kK = kQ + kLanes * kTileBytes;
+  static constexpr int kV = kK + kLanes * kTileBytes;
+  static constexpr int kEnt = kV + kLanes * kTileBytes;     // lane x at + x * entries
+  static constexpr int kBm = kEnt + kLanes * kAttnMaxEntries * 4;
   static constexpr int kScan = kBm + 2 * kAttnMaxBitmapWords * 4;
   static constexpr int kBar = kScan + kAttnMaxBitmapWords * 4;
-  static constexpr int kMisc = kBar + 16 * 8;
+  static constexpr int kMisc = kBar + 32 * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
 };
 
-// Barrier slots (each completes once per key tile, except Q and drain).
+// Barrier slots of lane x: 8 * x + slot.
 enum : int { kBarQ = 0, kBarKFull = 1, kBarVFull = 2, kBarKEmpty = 3, kBarVEmpty = 4, kBarSFull = 5,
-             kBarPFull = 6, kBarO = 7, kBarDrain = 8 };
+             kBarPFull = 6, kBarODone = 7 };
+constexpr int kBarDrain = 16;
 
 // Above this growth of the row maximum (log2 units) O is rescaled; below
 // it the stale maximum is kept, so P <= 2^8.
@@ -71,35 +79,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-// (a * b + c) on a pair of floats in one packed instruction.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
 }
 
 // A wait with its own limit that ignores the abort flag (used while draining).
@@ -223,185 +202,254 @@ __device__ int build_units(const AttnArgs& a, int m, int bh, uint32_t* ents, uin
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__device__ __forceinline__ void issue_s(uint32_t s_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = (uint32_t)((k >> 2) * AttnSmem<D>::kChunkBytes + (k & 3) * 32);
+    mma_ss(s_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+           kIdS, k > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         bool accumulate) {
+  constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, 0, 1);    // P (tmem), V MN-major
+#pragma unroll
+  for (int k = 0; k < kBN / 16; ++k) {
+    mma_ts(o_tmem, p_tmem + (uint32_t)(k * 8),
+           smem_desc_sw128(v_addr + (uint32_t)(k * 2048), AttnSmem<D>::kChunkBytes, 1024), kIdO,
+           (accumulate || k > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using L = AttnSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int m = blockIdx.x;
   const int bh = blockIdx.y;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int* total_slot = reinterpret_cast<int*>(smem + L::kMisc + 8);
+  int m_of[kLanes];
+  for (int x = 0; x < kLanes; ++x) m_of[x] = kLanes * blockIdx.x + x;
 
   if (tid == 0) {
-    mbar_init(&bar[kBarQ], 1);
-    mbar_init(&bar[kBarKFull], 1);
-    mbar_init(&bar[kBarVFull], 1);
-    mbar_init(&bar[kBarKEmpty], 1);
-    mbar_init(&bar[kBarVEmpty], 1);
-    mbar_init(&bar[kBarSFull], 1);
-    mbar_init(&bar[kBarPFull], 128);
-    mbar_init(&bar[kBarO], 1);
+    for (int x = 0; x < kLanes; ++x) {
+      uint64_t* b = bar + 8 * x;
+      mbar_init(&b[kBarQ], 1);
+      mbar_init(&b[kBarKFull], 1);
+      mbar_init(&b[kBarVFull], 1);
+      mbar_init(&b[kBarKEmpty], 1);
+      mbar_init(&b[kBarVEmpty], 1);
+      mbar_init(&b[kBarSFull], 1);
+      mbar_init(&b[kBarPFull], 128);
+      mbar_init(&b[kBarODone], 1);
+    }
     mbar_init(&bar[kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  const int E = build_units(a, m, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
-                            reinterpret_cast<uint32_t*>(smem + L::kScan), total_slot);
+  int N[kLanes];
+  for (int x = 0; x < kLanes; ++x) {
+    int E = 0;
+    if (m_of[x] < a.MT)
+      E = build_units(a, m_of[x], bh, reinterpret_cast<uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries,
+                      reinterpret_cast<uint32_t*>(smem + L::kBm), reinterpret_cast<uint32_t*>(smem + L::kScan),
+                      total_slot);
+    N[x] = E;  // units for now; tiles below
+  }
+  int E_of[kLanes];
+  for (int x = 0; x < kLanes; ++x) {
+    E_of[x] = N[x];
+    N[x] = (N[x] + 1) >> 1;  // 128-key tiles
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int N = (E + 1) >> 1;  // 128-key tiles
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // K(n) goes into the K slot once S(n-1) has consumed it; V(n) into the V
-    // slot once PV(n-1) has.
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
-      int k_issued = 0, v_issued = 0;
-      for (int n = 0; n < N; ++n) {
+      int k_issued[kLanes] = {0, 0}, v_issued[kLanes] = {0, 0};
+      auto load_kv = [&](int x, int n, bool is_v) {
+        const uint32_t* ents = reinterpret_cast<const uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries;
         const uint32_t e0 = ents[2 * n];
-        const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : (e0 & 0xFFFF0000u);
+        const uint32_t e1 = (2 * n + 1 < E_of[x]) ? ents[2 * n + 1] : (e0 & 0xFFFF0000u);
         const int r0 = (int)(e0 >> 16) * 64;
         const int r1 = (int)(e1 >> 16) * 64;
-        if (n >= 1 && !mbar_wait(&bar[kBarKEmpty], (n - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(&bar[kBarKFull], L::kTileBytes);
+        uint64_t* full = &bar[8 * x + (is_v ? kBarVFull : kBarKFull)];
+        uint8_t* dst = smem + (is_v ? L::kV : L::kK) + x * L::kTileBytes;
+        const CUtensorMap* map = is_v ? &tmV : &tmK;
+        mbar_arrive_expect_tx(full, L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(smem + L::kK + c * L::kChunkBytes, &tmK, &bar[kBarKFull], c * 64, r0, bh);
-          tma_load_3d(smem + L::kK + c * L::kChunkBytes + 8192, &tmK, &bar[kBarKFull], c * 64, r1, bh);
+          tma_load_3d(dst + c * L::kChunkBytes, map, full, c * 64, r0, bh);
+          tma_load_3d(dst + c * L::kChunkBytes + 8192, map, full, c * 64, r1, bh);
         }
-        k_issued = n + 1;
-        if (n >= 1 && !mbar_wait(&bar[kBarVEmpty], (n - 1) & 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(&bar[kBarVFull], L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(smem + L::kV + c * L::kChunkBytes, &tmV, &bar[kBarVFull], c * 64, r0, bh);
-          tma_load_3d(smem + L::kV + c * L::kChunkBytes + 8192, &tmV, &bar[kBarVFull], c * 64, r1, bh);
+      };
+      bool ok = true;
+      for (int x = 0; x < kLanes; ++x) {
+        if (N[x] == 0) continue;
+        mbar_arrive_expect_tx(&bar[8 * x + kBarQ], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(smem + L::kQ + x * L::kTileBytes + c * L::kChunkBytes, &tmQ, &bar[8 * x + kBarQ],
+                      c * 64, m_of[x] * kBM, bh);
+        load_kv(x, 0, false);
+        k_issued[x] = 1;
+        load_kv(x, 0, true);
+        v_issued[x] = 1;
+      }
+      const int n_max = N[0] > N[1] ? N[0] : N[1];
+      for (int n = 1; ok && n < n_max; ++n) {
+        // K of tile n once S(n-1) completed, then V once PV(n-1) completed,
+        // lane A before lane B: the order in which those events happen.
+        for (int x = 0; ok && x < kLanes; ++x) {
+          if (n >= N[x]) continue;
+          if (!mbar_wait(&bar[8 * x + kBarKEmpty], (n - 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          load_kv(x, n, false);
+          k_issued[x] = n + 1;
         }
-        v_issued = n + 1;
+        for (int x = 0; ok && x < kLanes; ++x) {
+          if (n >= N[x]) continue;
+          if (!mbar_wait(&bar[8 * x + kBarVEmpty], (n - 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          load_kv(x, n, true);
+          v_issued[x] = n + 1;
+        }
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
-        mbar_wait_drain(&bar[kBarQ], 0);
-        if (k_issued) mbar_wait_drain(&bar[kBarKFull], (k_issued - 1) & 1);
-        if (v_issued) mbar_wait_drain(&bar[kBarVFull], (v_issued - 1) & 1);
+        for (int x = 0; x < kLanes; ++x) {
+          if (N[x] == 0) continue;
+          mbar_wait_drain(&bar[8 * x + kBarQ], 0);
+          if (k_issued[x]) mbar_wait_drain(&bar[8 * x + kBarKFull], (k_issued[x] - 1) & 1);
+          if (v_issued[x]) mbar_wait_drain(&bar[8 * x + kBarVFull], (v_issued[x] - 1) & 1);
+        }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
-      constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, 0, 1);    // P (tmem), V MN-major
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
-      bool ok = mbar_wait(&bar[kBarQ], 0, abort_flag, a.err);
-      for (int n = 0; ok && n < N; ++n) {
-        const uint32_t par = n & 1;
-        if (!mbar_wait(&bar[kBarKFull], par, abort_flag, a.err)) break;
-        // P(n-1) lives in the S columns and O must be final before rescaling:
-        // PV(n-1) has to complete before S(n) is issued.
-        if (n >= 1 && !mbar_wait(&bar[kBarO], (n - 1) & 1, abort_flag, a.err)) break;
+      bool ok = true;
+      for (int x = 0; ok && x < kLanes; ++x) {
+        if (N[x] == 0) continue;
+        uint64_t* b = bar + 8 * x;
+        ok = mbar_wait(&b[kBarQ], 0, abort_flag, a.err) && mbar_wait(&b[kBarKFull], 0, abort_flag, a.err);
+        if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (uint32_t)((k >> 2) * L::kChunkBytes + (k & 3) * 32);
-          mma_ss(tmem, smem_desc_sw128(q_addr + off, 16, 1024),
-                 smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
+        issue_s<D>(tmem + 256u * x, q_addr + x * L::kTileBytes, k_addr + x * L::kTileBytes);
+        mma_commit(&b[kBarSFull]);
+        mma_commit(&b[kBarKEmpty]);
+      }
+      int np[kLanes] = {0, 0};
+      while (ok && (np[0] < N[0] || np[1] < N[1])) {
+        for (int x = 0; ok && x < kLanes; ++x) {
+          const int n = np[x];
+          if (n >= N[x]) continue;
+          uint64_t* b = bar + 8 * x;
+          if (!mbar_wait(&b[kBarPFull], n & 1, abort_flag, a.err) ||
+              !mbar_wait(&b[kBarVFull], n & 1, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D>(tmem + 256u * x + kOCol, tmem + 256u * x, v_addr + x * L::kTileBytes, n > 0);
+          mma_commit(&b[kBarVEmpty]);
+          if (n + 1 == N[x]) mma_commit(&b[kBarODone]);  // O final: the epilogue's single wait
+          np[x] = n + 1;
+          if (n + 1 < N[x]) {
+            // S(n+1) overwrites the columns holding P(n); PV(n) was issued
+            // before it by this thread and tcgen05.mma executes in issue
+            // order. Its commit also covers PV(n): once S(n+1) is reported
+            // complete, O holds PV(0..n) and may be rescaled.
+            if (!mbar_wait(&b[kBarKFull], (n + 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            tc_fence_after();
+            issue_s<D>(tmem + 256u * x, q_addr + x * L::kTileBytes, k_addr + x * L::kTileBytes);
+            mma_commit(&b[kBarSFull]);
+            mma_commit(&b[kBarKEmpty]);
+          }
         }
-        mma_commit(&bar[kBarSFull]);
-        mma_commit(&bar[kBarKEmpty]);
-        if (!mbar_wait(&bar[kBarPFull], par, abort_flag, a.err)) break;
-        if (!mbar_wait(&bar[kBarVFull], par, abort_flag, a.err)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          mma_ts(tmem + kOCol, tmem + (uint32_t)(k * 8),
-                 smem_desc_sw128(v_addr + (uint32_t)(k * 2048), L::kChunkBytes, 1024), kIdO,
-                 (n > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(&bar[kBarO]);
-        mma_commit(&bar[kBarVEmpty]);
       }
       mma_commit(&bar[kBarDrain]);
       mbar_wait_drain(&bar[kBarDrain], 0);
     }
-  } else {
+  } else if (warp < kLanes * 4) {
     // ------------------------------------------------------------ softmax
     const Dims& d = a.d;
-    const int r = tid;  // query row of the tile = TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int x = warp >> 2;           // lane (query tile) of this warp group
+    const int r = tid & 127;           // query row of the tile = TMEM lane
+    const int Nx = N[x];
+    const int Ex = E_of[x];
+    const uint32_t* ents = reinterpret_cast<const uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries;
+    uint64_t* b = bar + 8 * x;
+    const uint32_t trow = tmem + 256u * x + ((uint32_t)((warp & 3) * 32) << 16);
     const int qsel = r >> 6;   // warp-uniform
     const float sc = a.scale_log2;
     float m_used = -INFINITY;  // running maximum in scaled log2 units (possibly stale by < 8)
     float l_run = 0.f;
-    bool ok = true;
-    for (int n = 0; n < N; ++n) {
-      ok = mbar_wait(&bar[kBarSFull], n & 1, abort_flag, a.err);
+    bool ok = Nx > 0;
+    for (int n = 0; ok && n < Nx; ++n) {
+      ok = mbar_wait(&b[kBarSFull], n & 1, abort_flag, a.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(trow + (uint32_t)(32 * i), s[i]);
       const uint32_t e0 = ents[2 * n];
-      const uint32_t e1 = (2 * n + 1 < E) ? ents[2 * n + 1] : 0u;
+      const uint32_t e1 = (2 * n + 1 < Ex) ? ents[2 * n + 1] : 0u;
       const int lim0 = ((e0 >> qsel) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
       const int lim1 = ((e1 >> qsel) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
       const bool full = (lim0 == 64) && (lim1 == 64);   // warp-uniform
-
-      // pass 1: row maximum of the raw scores over the valid columns
-      float mx = -INFINITY;
+      tmem_wait_ld();
+      if (!full) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(trow + (uint32_t)(64 * h), s0);
-        tmem_ld32(trow + (uint32_t)(64 * h + 32), s1);
-        tmem_wait_ld();
-        const int lim = h == 0 ? lim0 : lim1;
-        if (full) {
+        for (int i = 0; i < 4; ++i) {
+          const int lim = i < 2 ? lim0 - 32 * i : lim1 - 32 * (i - 2);
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            mx = max3f(mx, __uint_as_float(s0[c]), __uint_as_float(s0[c + 1]));
-            mx = max3f(mx, __uint_as_float(s1[c]), __uint_as_float(s1[c + 1]));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c < lim) mx = fmaxf(mx, __uint_as_float(s0[c]));
-            if (c + 32 < lim) mx = fmaxf(mx, __uint_as_float(s1[c]));
-          }
+          for (int c = 0; c < 32; ++c)
+            if (c >= lim) s[i][c] = __float_as_uint(-INFINITY);
         }
       }
-      const float mt = mx * sc;  // -inf when nothing is valid
+      float ma = -INFINITY, mb = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          ma = max3f(ma, __uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1]));
+          mb = max3f(mb, __uint_as_float(s[i][c + 2]), __uint_as_float(s[i][c + 3]));
+        }
+      }
+      const float mt = fmaxf(ma, mb) * sc;  // -inf when nothing is valid
       const bool need = mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt > -INFINITY);
       if (__any_sync(0xFFFFFFFFu, need)) {
         const float m_new = need ? mt : m_used;
         const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
         if (n > 0) {
-          // O holds PV(0..n-1) (complete: S(n) was issued after PV(n-1)).
-#pragma unroll
-          for (int i = 0; i < D / 32; ++i) {
-            uint32_t o[32];
-            tmem_ld32(trow + kOCol + (uint32_t)(32 * i), o);
+          // O holds PV(0..n-1): the commit of S(n) covered PV(n-1).
+#pragma unroll 1
+          for (int i = 0; i < D / 16; ++i) {
+            uint32_t o[16];
+            tmem_ld16(trow + kOCol + (uint32_t)(16 * i), o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(trow + kOCol + (uint32_t)(32 * i), o);
+            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st16(trow + kOCol + (uint32_t)(16 * i), o);
           }
         }
         l_run *= alpha;
@@ -410,57 +458,42 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
       const float2 sc2 = make_float2(sc, sc);
       const float2 nb2 = make_float2(-base, -base);
-
-      // pass 2: P = exp2(s * scale - base), row sum, bf16 P into the S columns
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(trow + (uint32_t)(64 * h), s0);
-        tmem_ld32(trow + (uint32_t)(64 * h + 32), s1);
-        tmem_wait_ld();
-        const int lim = h == 0 ? lim0 : lim1;
-        uint32_t pk[32];
+      for (int h = 0; h < 4; ++h) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float2 x0 = ffma2(make_float2(__uint_as_float(s0[c]), __uint_as_float(s0[c + 1])), sc2, nb2);
-          float2 x1 = ffma2(make_float2(__uint_as_float(s1[c]), __uint_as_float(s1[c + 1])), sc2, nb2);
-          if (!full) {
-            if (c >= lim) x0.x = -INFINITY;
-            if (c + 1 >= lim) x0.y = -INFINITY;
-            if (c + 32 >= lim) x1.x = -INFINITY;
-            if (c + 33 >= lim) x1.y = -INFINITY;
-          }
-          const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
-          const float2 p1 = make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
-          acc0 = fadd2(acc0, p0);
-          acc1 = fadd2(acc1, p1);
-          pk[c >> 1] = cvt_bf16x2(p0.x, p0.y);
-          pk[16 + (c >> 1)] = cvt_bf16x2(p1.x, p1.y);
+        for (int q = 0; q < 16; ++q) {
+          const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
+                                  sc2, nb2);
+          const float2 p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
+          if (q & 1) acc1 = fadd2(acc1, p);
+          else acc0 = fadd2(acc0, p);
+          pk[q] = cvt_bf16x2(p.x, p.y);
         }
-        tmem_st32(trow + (uint32_t)(32 * h), pk);
+        tmem_st16(trow + (uint32_t)(16 * h), pk);
       }
       l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[kBarPFull]);
+      mbar_arrive(&b[kBarPFull]);
     }
     // ------------------------------------------------------------ epilogue
     if (ok) {
-      ok = mbar_wait(&bar[kBarO], (N - 1) & 1, abort_flag, a.err);
+      ok = mbar_wait(&b[kBarODone], 0, abort_flag, a.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
     }
     if (ok) {
       tc_fence_after();
-      const int pr = m * kBM + r;  // row in the padded chunk
+      const int pr = m_of[x] * kBM + r;  // row in the padded chunk
       const int f = pr / d.T_pad;
       const int rr = pr - f * d.T_pad;
       const bool row_ok = (f < d.Fc) && (rr < d.T_f);
-      const int b = bh / d.H;
-      const int h = bh - b * d.H;
+      const int bb = bh / d.H;
+      const int h = bh - bb * d.H;
       const size_t n_tok = (size_t)f * d.T_f + rr;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      uint16_t* orow = a.out + (((size_t)b * d.Lq + n_tok) * d.H + h) * D;
+      uint16_t* orow = a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D;
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
         uint32_t o[32];
@@ -484,7 +517,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -528,7 +561,7 @@ static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.MT, a.d.B * a.d.H);
+  dim3 grid((a.MT + kLanes - 1) / kLanes, a.d.B * a.d.H);
   attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
