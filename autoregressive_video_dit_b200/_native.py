@@ -82,6 +82,8 @@ _SIGS = {
     "cva_chunk_attention": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
                                       c_int32, c_int32, c_int32, c_void_p, c_size_t, c_void_p,
                                       c_void_p, c_void_p]),
+    "cva_chunk_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
+                                              c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
     "cva_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
     "cva_kv_cache_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
@@ -306,3 +308,12 @@ def chunk_attention(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0:
     check(lib.cva_chunk_attention(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
                                   ctypes.byref(tables.struct), t0, k_f, k_b, _ptr(workspace),
                                   ws_bytes, _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def chunk_attention_noalloc(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, k_f: int,
+                            k_b: int, out, lse=None, stream=None) -> None:
+    """chunk_attention with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate device memory; see cva.h)."""
+    check(lib.cva_chunk_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
+                                          ctypes.byref(tables.struct), t0, k_f, k_b, _ptr(out),
+                                          _ptr(lse), _stream(stream)))

@@ -163,6 +163,10 @@ int check_attn_limits(const Dims& d, int F, bool dense, int k_b_max) {
 
 }  // namespace
 
+namespace cva {
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace cva
+
 extern "C" {
 
 int cva_version(void) { return CVA_VERSION; }

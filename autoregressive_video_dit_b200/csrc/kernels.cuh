@@ -74,6 +74,9 @@ constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
 cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
                              const void* cache_v, cudaStream_t stream, const char** why);
 
+// Sets the thread-local message cva_last_error() returns; returns `code`.
+int report_error(int code, const char* msg);
+
 // ---- diagnostics (diag.cu) ------------------------------------------------
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 

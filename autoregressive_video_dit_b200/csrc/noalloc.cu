@@ -1,0 +1,74 @@
+// cva_chunk_attention_noalloc: the fused chunk call for callers that cannot
+// allocate device memory when they call it -- for example a plugin inside a
+// host runtime that owns every allocation and hands the plugin only its
+// input and output buffers, or a real-time loop that forbids allocation
+// after start-up. Instead of a caller-provided workspace it uses one fixed
+// scratch array in this file, reserved on every device that loads the
+// library for as long as the process lives.
+#include <stdio.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace {
+
+// Fixed scratch: enough for the 1.3B-shaped 480P chunk (H = 12, D = 128,
+// 30 x 52 latent grid, 3 frames per chunk) with any budget up to 1024
+// candidate blocks; larger shapes are rejected.
+constexpr size_t kNoAllocScratchBytes = 24u << 20;  // 24 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// The array's name is only a host-side stand-in; its device address is
+// looked up once per device, with that device current, and cached.
+void* noalloc_scratch_address(int* rc) {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 128) {
+    *rc = cva::report_error(CVA_ELAUNCH, "noalloc: cannot query the current device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      char msg[256];
+      snprintf(msg, sizeof(msg), "noalloc: cudaGetSymbolAddress of the fixed scratch failed: %s",
+               cudaGetErrorString(e));
+      *rc = cva::report_error(CVA_ELAUNCH, msg);
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *rc = CVA_OK;
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" int cva_chunk_attention_noalloc(const void* q, const void* k, const void* v,
+                                           const cva_kv_cache* cache, const cva_rope_tables* tables,
+                                           int32_t t0, int32_t k_f, int32_t k_b, void* out, float* lse,
+                                           cva_stream_t stream) {
+  if (!cache) return cva::report_error(CVA_EINVAL, "cache is NULL");
+  size_t need = 0;
+  int rc = cva_chunk_workspace_bytes(&cache->shape, k_f, k_b, &need);
+  if (rc) return rc;
+  if (need > kNoAllocScratchBytes) {
+    char msg[256];
+    snprintf(msg, sizeof(msg),
+             "noalloc: this shape and budget need %zu bytes of scratch; the fixed scratch holds %zu "
+             "(use cva_chunk_attention with a caller workspace)",
+             need, kNoAllocScratchBytes);
+    return cva::report_error(CVA_ENOMEM, msg);
+  }
+  void* ws = noalloc_scratch_address(&rc);
+  if (!ws) return rc;
+  // Nothing in the workspace has to start at zero: every byte the path reads
+  // is written earlier in the same call.
+  return cva_chunk_attention(q, k, v, cache, tables, t0, k_f, k_b, ws, kNoAllocScratchBytes, out, lse,
+                             stream);
+}

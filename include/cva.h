@@ -244,6 +244,24 @@ int cva_chunk_attention(const void* q, const void* k, const void* v,
                         int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
                         size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
+/* The fused chunk call without a caller workspace (the pages have no
+ * counterpart; this exists for callers that cannot allocate device memory
+ * when they call, such as a plugin whose host runtime owns every allocation
+ * and passes it only inputs and outputs, or a loop that forbids allocation
+ * after start-up). Same arguments and results as cva_chunk_attention; the
+ * scratch is one fixed 24 MiB array inside the library, held on every
+ * device that loads it until the process exits. Shapes and budgets that
+ * need more return CVA_ENOMEM without launching. Calls never allocate or
+ * free memory. The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress), so make it before any stream capture. All calls
+ * share the one array and keep whatever the last call left in it: calls
+ * that overlap on the GPU (different streams, or different host threads on
+ * one device) race on it, so order them on one stream. */
+int cva_chunk_attention_noalloc(const void* q, const void* k, const void* v,
+                                const cva_kv_cache* cache, const cva_rope_tables* tables,
+                                int32_t t0, int32_t k_f, int32_t k_b, void* out, float* lse,
+                                cva_stream_t stream);
+
 /* Per-stage timing of cva_chunk_attention on this host thread: while set,
  * each call records events[0] before its first launch, events[1] after the
  * rotate/append/pool kernels, events[2] after the selection (right after
