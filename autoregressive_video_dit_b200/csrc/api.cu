@@ -150,14 +150,16 @@ int check_attn_limits(const Dims& d, int F, bool dense, int k_b_max) {
     if ((int64_t)F * d.nb > 32 * kAttnMaxBitmapWords)
       return fail(CVA_ENOTSUP, "history blocks %lld exceed %d for the sparse attention",
                   (long long)F * d.nb, 32 * kAttnMaxBitmapWords);
+    // a query tile holds nq query blocks (two when blk = 64)
     const int nq = d.blk == 64 ? 2 : 1;
     int64_t u = (int64_t)nq * k_b_max;
     if (u > (int64_t)F * d.nb) u = (int64_t)F * d.nb;
     hist = u * upb;
   }
-  if (hist + cur > kAttnMaxEntries)
-    return fail(CVA_ENOTSUP, "key units per query tile %lld exceed %d", (long long)(hist + cur),
-                kAttnMaxEntries);
+  // + one padding unit per section
+  if (hist + cur + 3 > kAttnMaxEntries)
+    return fail(CVA_ENOTSUP, "key units per query tile %lld exceed %d",
+                (long long)(hist + cur + 3), kAttnMaxEntries);
   return CVA_OK;
 }
 

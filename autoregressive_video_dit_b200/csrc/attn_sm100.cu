@@ -4,30 +4,35 @@
 // picked frame-block pairs, here together with every token of the current
 // chunk; its cost is independent of how long the history is.
 //
-// A CTA owns one SM and works on two 128-row query tiles of one (batch,
-// head) at once, in two independent lanes (A and B). Each lane has its own
-// key list, its own Q, K and V tiles in shared memory and its own S and O
-// accumulators in tensor memory (4 x 128 columns). A key list is a list of
-// 64-row key units: the union of the picked history blocks of the lane's
-// query blocks (two 64-token query blocks share a tile when blk = 64; a unit
-// carries a 2-bit mask of the query blocks that picked it), followed by the
-// current chunk's blocks. Pairs of units form 128-key tiles.
+// A CTA owns one SM and one 128-row query tile of one (batch, head). Its
+// keys come as a stream of 64-row key units, two per 128-key tile: the
+// current chunk's blocks, then the union of the history blocks its query
+// blocks picked (two 64-token query blocks share a tile when blk = 64; a
+// unit's mask says which of them picked it); an odd count is padded with an
+// empty unit.
+//
+// Tensor memory holds two score buffers S0 and S1 (128 fp32 columns each,
+// P aliased onto the scores it came from) and the output accumulator O
+// (128 columns). With two score buffers the tensor core computes S(i+1)
+// while the softmax works on S(i), and PV(i) is followed right away by
+// S(i+2) into the buffer P(i) leaves: the MMAs of one tile overlap the
+// softmax of the next instead of waiting for it.
 //
 // Roles (384 threads):
-//   warps 0-3 / 4-7: softmax of lane A / B; thread i owns query row i
-//     (TMEM lane i). One tensor-memory load brings the 128 scores of a tile
-//     into registers; masks, row maximum (3-input max), exp2 on the MUFU in
-//     fp32 with packed f32x2 arithmetic, bf16 P written back over the S
-//     columns. O is rescaled in tensor memory only when the row maximum grows
-//     by more than 2^8. Finally O is normalised into bf16.
-//   warp 8 (one lane): TMA producer. Q once per lane; then per key tile K
-//     into the lane's K slot (free once S of the previous tile completed) and
-//     V into its V slot (free once PV completed), gathered by block index
-//     with one 64-row box per unit and 64-column chunk, 128-byte swizzle.
-//     No multicast.
-//   warp 9 (one lane): tcgen05.mma issuer, interleaving the lanes:
-//     PV_A(n), S_A(n+1), PV_B(n), S_B(n+1), ... so that one lane's MMAs run
-//     while the other lane's softmax does.
+//   warps 0-7: softmax. Warps w and w + 4 own query rows 32 (w mod 4) ..
+//     + 31 (TMEM lanes; thread = row) and split the 128 key columns: warp
+//     w < 4 the first 64, warp w + 4 the last 64. They trade partial row
+//     maxima through shared memory (one named barrier per warp pair), then
+//     exp2 on the MUFU in fp32 with packed f32x2 arithmetic and write bf16 P
+//     over the S columns. O is rescaled in tensor memory only when the row
+//     maximum grows by more than 2^8, after PV(i-1) completed. Finally each
+//     warp normalises its half of O into bf16.
+//   warp 8 (one lane): TMA producer. Q once, then K and V of every tile in
+//     order into the ring slot t mod 2, each as soon as its slot is free,
+//     gathered by block index with one 64-row box per unit and 64-column
+//     chunk, 128-byte swizzle. No multicast.
+//   warp 9 (one lane): tcgen05.mma issuer, in the fixed order S(0), S(1),
+//     PV(0), S(2), PV(1), S(3), ...
 // Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
 // roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait and the tensor memory is released.
@@ -40,45 +45,58 @@ namespace cva {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kLanes = 2;
+constexpr int kStages = 2;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 // 12 warps: registers are granted per group of four warps, so warps 10 and
 // 11 cost nothing extra; they only join the final barrier.
 constexpr int kAttnThreads = 384;
-constexpr uint32_t kTmemCols = 512;   // lane x: S at 256x (P aliased onto it), O at 256x + 128
-constexpr uint32_t kOCol = 128;
+constexpr uint32_t kTmemCols = 512;   // S0 at 0, S1 at 128, O at 256
+constexpr uint32_t kOCol = 256;
 
 template <int D>
 struct AttnSmem {
   static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B: one 64-column chunk
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // a Q, K or V tile
-  static constexpr int kQ = 0;                              // lane x at + x * tile
-  static constexpr int kK = kQ + kLanes * kTileBytes;
-  static constexpr int kV = kK + kLanes * kTileBytes;
-  static constexpr int kEnt = kV + kLanes * kTileBytes;     // lane x at + x * entries
-  static constexpr int kBm = kEnt + kLanes * kAttnMaxEntries * 4;
-  static constexpr int kScan = kBm + 2 * kAttnMaxBitmapWords * 4;
-  static constexpr int kBar = kScan + kAttnMaxBitmapWords * 4;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;                // slot s at + s * tile
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kEnt = kV + kStages * kTileBytes;
+  // softmax pair exchange: maxima [2 bufs][2 halves][128], sums [2][128], flags [3][2][4]
+  static constexpr int kRed = kEnt + kAttnMaxEntries * 4;
+  static constexpr int kBar = kRed + (2 * 2 * 128 + 2 * 128) * 4 + 3 * 2 * 4 * 4;
   static constexpr int kMisc = kBar + 32 * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
+  // While the key list is built, its bitmaps and counts live in the V ring.
+  static constexpr int kBm = kV;                                   // 4 bitmaps
+  static constexpr int kCnt = kBm + 4 * kAttnMaxBitmapWords * 4;   // 3 count arrays
+  static_assert(7 * kAttnMaxBitmapWords * 4 <= kStages * kTileBytes, "build scratch");
 };
 
-// Barrier slots of lane x: 8 * x + slot.
-enum : int { kBarQ = 0, kBarKFull = 1, kBarVFull = 2, kBarKEmpty = 3, kBarVEmpty = 4, kBarSFull = 5,
-             kBarPFull = 6, kBarODone = 7 };
-constexpr int kBarDrain = 16;
+// Barriers: S buffer b full / P written into it; K and V ring slots full and
+// free; PV done (every PV), O final; one for draining the tensor pipe.
+constexpr int kBarSFull = 0, kBarPFull = 2, kBarKFull = 4, kBarKEmpty = 6, kBarVFull = 8,
+              kBarVEmpty = 10, kBarQ = 12, kBarPVDone = 13, kBarODone = 14, kBarDrain = 15;
 
 // Above this growth of the row maximum (log2 units) O is rescaled; below
 // it the stale maximum is kept, so P <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
 
+// Longest sleep of the idle producer on one barrier (ns).
+constexpr uint32_t kSleepNs = 1000;
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Barrier of the two warps that share a row range (ids 1..4; 0 is __syncthreads).
+__device__ __forceinline__ void pair_sync(int quarter) {
+  asm volatile("bar.sync %0, 64;" ::"r"(quarter + 1) : "memory");
 }
 
 // A wait with its own limit that ignores the abort flag (used while draining).
@@ -90,7 +108,8 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 }
 
 // Key unit: (row64 << 16) | (valid << 8) | mask. row64 indexes 64-row
-// groups inside one (batch, head) slice of the cache.
+// groups inside one (batch, head) slice of the cache; an empty unit (row 0,
+// valid 0, mask 0) pads a section to whole tiles.
 __device__ __forceinline__ uint32_t make_unit(int row64, int valid, uint32_t mask) {
   return ((uint32_t)row64 << 16) | ((uint32_t)valid << 8) | mask;
 }
@@ -100,105 +119,151 @@ __device__ __forceinline__ int unit_valid(int block_valid, int u) {
   return v < 0 ? 0 : (v > 64 ? 64 : v);
 }
 
-// Builds the tile's key-unit list in smem; returns the number of units.
-// Must be called by all threads of the CTA.
-__device__ int build_units(const AttnArgs& a, int m, int bh, uint32_t* ents, uint32_t* bm,
-                           uint32_t* wcnt, int* total_slot) {
+// Tile counts of a key stream (one query tile, or two sharing the stream).
+struct Stream {
+  int TS;    // shared tiles (both lanes)
+  int TA;    // lane A only
+  int TB;    // lane B only
+  int mn;    // min(TA, TB): interleaved pairs
+  __device__ __forceinline__ int total() const { return TS + TA + TB; }
+  __device__ __forceinline__ int tiles_of(int x) const { return TS + (x == 0 ? TA : TB); }
+  // Stream position of lane x's i-th tile.
+  __device__ __forceinline__ int tile_of(int x, int i) const {
+    if (i < TS) return i;
+    const int k = i - TS;
+    return TS + (k < mn ? 2 * k + x : mn + k);
+  }
+  // Entry index of the i-th unit of lane x's private list.
+  __device__ __forceinline__ int private_entry(int x, int i) const {
+    return 2 * tile_of(x, TS + (i >> 1)) + (i & 1);
+  }
+};
+
+// Builds the key stream of the CTA's lanes (tile m0 and, if has_b, m0 + 1)
+// into `ents`; must be called by all threads of the CTA.
+__device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, uint32_t* ents,
+                               uint32_t* bm, uint32_t* cnt, int* tot) {
+  constexpr int kW = kAttnMaxBitmapWords;
   const Dims& d = a.d;
   const int tid = threadIdx.x;
   const int upb = d.blk / 64;
   const int rows64_slot = d.T_pad / 64;
-  int hist = 0;
-  if (a.F > 0) {
-    if (a.block_idx == nullptr) {
-      hist = a.F * d.nb * upb;
-      for (int i = tid; i < hist; i += kAttnThreads) {
-        const int br = i / upb, u = i - br * upb;
-        const int fp = br / d.nb, j = br - fp * d.nb;
-        const int slot = (a.t_lo + fp) % a.W;
-        const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-        ents[i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 3u);
-      }
-    } else {
-      const int nbits = a.F * d.nb;
-      const int nw = (nbits + 31) >> 5;
-      for (int i = tid; i < nw; i += kAttnThreads) {
-        bm[i] = 0u;
-        bm[kAttnMaxBitmapWords + i] = 0u;
-      }
-      __syncthreads();
-      const int nq = (d.blk == 64) ? 2 : 1;
+  const uint32_t all_mask = has_b ? 0xFu : 0x3u;
+  const int nbits = a.F * d.nb;
+  const int nw = (nbits + 31) >> 5;
+  const bool sparse = a.F > 0 && a.block_idx != nullptr;
+  int nS = (a.F > 0 && !sparse) ? nbits * upb : 0, nA = 0, nB = 0;
+  if (sparse) {
+    for (int i = tid; i < 4 * nw; i += kAttnThreads) bm[(i / nw) * kW + i % nw] = 0u;
+    __syncthreads();
+    const int nq = (d.blk == 64) ? 2 : 1;
+    for (int x = 0; x < (has_b ? 2 : 1); ++x) {
       for (int q = 0; q < nq; ++q) {
-        const int qb = (d.blk == 64) ? 2 * m + q : m;
+        const int qb = (d.blk == 64) ? 2 * (m0 + x) + q : m0 + x;
         if (qb >= d.NQB) continue;
         const size_t u = (size_t)bh * d.NQB + qb;
-        int cnt = a.block_cnt ? a.block_cnt[u] : a.k_b_max;
-        if (cnt < 0 || cnt > a.k_b_max) {
+        int c = a.block_cnt ? a.block_cnt[u] : a.k_b_max;
+        if (c < 0 || c > a.k_b_max) {
           if (tid == 0) latch_error(a.err, CVA_DEV_BAD_COUNT);
-          cnt = cnt < 0 ? 0 : a.k_b_max;
+          c = c < 0 ? 0 : a.k_b_max;
         }
         const int32_t* lst = a.block_idx + u * a.k_b_max;
-        for (int i = tid; i < cnt; i += kAttnThreads) {
+        uint32_t* row = bm + (2 * x + q) * kW;
+        for (int i = tid; i < c; i += kAttnThreads) {
           const int id = lst[i];
           const int rel = id - a.t_lo * d.nb;
           if (id < 0 || rel < 0 || rel >= nbits) {
             latch_error(a.err, CVA_DEV_BAD_INDEX);
             continue;
           }
-          atomicOr(&bm[q * kAttnMaxBitmapWords + (rel >> 5)], 1u << (rel & 31));
+          atomicOr(&row[rel >> 5], 1u << (rel & 31));
+          if (nq == 1) atomicOr(&row[kW + (rel >> 5)], 1u << (rel & 31));  // both bits of the lane
         }
       }
-      __syncthreads();
-      for (int w = tid; w < nw; w += kAttnThreads)
-        wcnt[w] = __popc(bm[w] | bm[kAttnMaxBitmapWords + w]) * upb;
-      __syncthreads();
-      if (tid < 32) {  // exclusive scan of the per-word counts
-        int carry = 0;
-        for (int base = 0; base < nw; base += 32) {
-          const int w = base + tid;
-          const int v = (w < nw) ? (int)wcnt[w] : 0;
-          int incl = v;
+    }
+    __syncthreads();
+    for (int w = tid; w < nw; w += kAttnThreads) {
+      const uint32_t ia = bm[w] | bm[kW + w], ib = bm[2 * kW + w] | bm[3 * kW + w];
+      cnt[w] = __popc(ia & ib) * upb;
+      cnt[kW + w] = __popc(ia & ~ib) * upb;
+      cnt[2 * kW + w] = __popc(ib & ~ia) * upb;
+    }
+    __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < 3) {  // exclusive scan of class `warp`'s per-word counts
+      uint32_t* c = cnt + warp * kW;
+      int carry = 0;
+      for (int base = 0; base < nw; base += 32) {
+        const int w = base + lane;
+        const int v = (w < nw) ? (int)c[w] : 0;
+        int incl = v;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (tid >= o) incl += t;
-          }
-          if (w < nw) wcnt[w] = (uint32_t)(carry + incl - v);
-          carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += t;
         }
-        if (tid == 0) *total_slot = carry;
+        if (w < nw) c[w] = (uint32_t)(carry + incl - v);
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
       }
-      __syncthreads();
-      hist = *total_slot;
-      for (int w = tid; w < nw; w += kAttnThreads) {
-        const uint32_t b0 = bm[w], b1 = bm[kAttnMaxBitmapWords + w];
-        uint32_t any = b0 | b1;
-        int pos = (int)wcnt[w];
-        while (any) {
-          const int bit = __ffs(any) - 1;
-          any &= any - 1u;
-          const int rel = w * 32 + bit;
-          const int fp = rel / d.nb, j = rel - fp * d.nb;
-          const int slot = (a.t_lo + fp) % a.W;
-          const uint32_t mask =
-              (d.blk == 64) ? (((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1)) : 3u;
-          const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-          for (int u = 0; u < upb; ++u)
-            ents[pos++] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
+      if (lane == 0) tot[warp] = carry;
+    }
+    __syncthreads();
+    nS = tot[0];
+    nA = tot[1];
+    nB = tot[2];
+  }
+  const int cur = d.Fc * d.nb * upb;
+  Stream st;
+  st.TS = (nS + cur + 1) >> 1;
+  st.TA = (nA + 1) >> 1;
+  st.TB = (nB + 1) >> 1;
+  st.mn = st.TA < st.TB ? st.TA : st.TB;
+  if (a.F > 0 && !sparse) {
+    for (int i = tid; i < nS; i += kAttnThreads) {
+      const int br = i / upb, u = i - br * upb;
+      const int fp = br / d.nb, j = br - fp * d.nb;
+      const int slot = (a.t_lo + fp) % a.W;
+      const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+      ents[i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), all_mask);
+    }
+  } else if (sparse) {
+    for (int w = tid; w < nw; w += kAttnThreads) {
+      const uint32_t b0 = bm[w], b1 = bm[kW + w], b2 = bm[2 * kW + w], b3 = bm[3 * kW + w];
+      const uint32_t ia = b0 | b1, ib = b2 | b3;
+      uint32_t any = ia | ib;
+      int pos[3] = {(int)cnt[w], (int)cnt[kW + w], (int)cnt[2 * kW + w]};
+      while (any) {
+        const int bit = __ffs(any) - 1;
+        any &= any - 1u;
+        const int cls = ((ia >> bit) & 1u) ? (((ib >> bit) & 1u) ? 0 : 1) : 2;
+        const int rel = w * 32 + bit;
+        const int fp = rel / d.nb, j = rel - fp * d.nb;
+        const int slot = (a.t_lo + fp) % a.W;
+        const uint32_t mask = ((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1) | (((b2 >> bit) & 1u) << 2) |
+                              (((b3 >> bit) & 1u) << 3);
+        const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+        for (int u = 0; u < upb; ++u) {
+          const int i = pos[cls]++;
+          const int e = cls == 0 ? i : st.private_entry(cls - 1, i);
+          ents[e] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
         }
       }
     }
   }
-  const int cur = d.Fc * d.nb * upb;
   for (int i = tid; i < cur; i += kAttnThreads) {
     const int br = i / upb, u = i - br * upb;
     const int f = br / d.nb, j = br - f * d.nb;
     const int slot = (a.t0 + f) % a.W;
     const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-    ents[hist + i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 3u);
+    ents[nS + i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), all_mask);
+  }
+  if (tid == 0) {
+    if ((nS + cur) & 1) ents[2 * st.TS - 1] = 0u;
+    if (nA & 1) ents[st.private_entry(0, nA)] = 0u;
+    if (nB & 1) ents[st.private_entry(1, nB)] = 0u;
   }
   __syncthreads();
-  return hist + cur;
+  return st;
 }
 
 template <int D>
@@ -224,6 +289,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   }
 }
 
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -233,28 +299,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int bh = blockIdx.y;
+  const int m = blockIdx.x;  // query tile
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  int* total_slot = reinterpret_cast<int*>(smem + L::kMisc + 8);
-  int m_of[kLanes];
-  for (int x = 0; x < kLanes; ++x) m_of[x] = kLanes * blockIdx.x + x;
+  int* tot = reinterpret_cast<int*>(smem + L::kMisc + 8);  // 3 ints
+  uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
 
   if (tid == 0) {
-    for (int x = 0; x < kLanes; ++x) {
-      uint64_t* b = bar + 8 * x;
-      mbar_init(&b[kBarQ], 1);
-      mbar_init(&b[kBarKFull], 1);
-      mbar_init(&b[kBarVFull], 1);
-      mbar_init(&b[kBarKEmpty], 1);
-      mbar_init(&b[kBarVEmpty], 1);
-      mbar_init(&b[kBarSFull], 1);
-      mbar_init(&b[kBarPFull], 128);
-      mbar_init(&b[kBarODone], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[kBarSFull + s], 1);
+      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps);
+      mbar_init(&bar[kBarKFull + s], 1);
+      mbar_init(&bar[kBarKEmpty + s], 1);
+      mbar_init(&bar[kBarVFull + s], 1);
+      mbar_init(&bar[kBarVEmpty + s], 1);
     }
+    mbar_init(&bar[kBarQ], 1);
+    mbar_init(&bar[kBarPVDone], 1);
+    mbar_init(&bar[kBarODone], 1);
     mbar_init(&bar[kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -263,20 +329,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  int N[kLanes];
-  for (int x = 0; x < kLanes; ++x) {
-    int E = 0;
-    if (m_of[x] < a.MT)
-      E = build_units(a, m_of[x], bh, reinterpret_cast<uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries,
-                      reinterpret_cast<uint32_t*>(smem + L::kBm), reinterpret_cast<uint32_t*>(smem + L::kScan),
-                      total_slot);
-    N[x] = E;  // units for now; tiles below
-  }
-  int E_of[kLanes];
-  for (int x = 0; x < kLanes; ++x) {
-    E_of[x] = N[x];
-    N[x] = (N[x] + 1) >> 1;  // 128-key tiles
-  }
+  const Stream st = build_stream(a, m, false, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
+                                 reinterpret_cast<uint32_t*>(smem + L::kCnt), tot);
+  const int N = st.total();  // key tiles, in stream order
+  // the build scratch in the V ring is dead; the async proxy may now write it
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -288,15 +345,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int k_issued[kLanes] = {0, 0}, v_issued[kLanes] = {0, 0};
-      auto load_kv = [&](int x, int n, bool is_v) {
-        const uint32_t* ents = reinterpret_cast<const uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries;
-        const uint32_t e0 = ents[2 * n];
-        const uint32_t e1 = (2 * n + 1 < E_of[x]) ? ents[2 * n + 1] : (e0 & 0xFFFF0000u);
+      auto load_kv = [&](int t, bool is_v) {
+        const uint32_t e0 = ents[2 * t], e1 = ents[2 * t + 1];
         const int r0 = (int)(e0 >> 16) * 64;
         const int r1 = (int)(e1 >> 16) * 64;
-        uint64_t* full = &bar[8 * x + (is_v ? kBarVFull : kBarKFull)];
-        uint8_t* dst = smem + (is_v ? L::kV : L::kK) + x * L::kTileBytes;
+        const int s = t & 1;
+        uint64_t* full = &bar[(is_v ? kBarVFull : kBarKFull) + s];
+        uint8_t* dst = smem + (is_v ? L::kV : L::kK) + s * L::kTileBytes;
         const CUtensorMap* map = is_v ? &tmV : &tmK;
         mbar_arrive_expect_tx(full, L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c) {
@@ -304,42 +359,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_3d(dst + c * L::kChunkBytes + 8192, map, full, c * 64, r1, bh);
         }
       };
-      bool ok = true;
-      for (int x = 0; x < kLanes; ++x) {
-        if (N[x] == 0) continue;
-        mbar_arrive_expect_tx(&bar[8 * x + kBarQ], L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(smem + L::kQ + x * L::kTileBytes + c * L::kChunkBytes, &tmQ, &bar[8 * x + kBarQ],
-                      c * 64, m_of[x] * kBM, bh);
-        load_kv(x, 0, false);
-        k_issued[x] = 1;
-        load_kv(x, 0, true);
-        v_issued[x] = 1;
-      }
-      const int n_max = N[0] > N[1] ? N[0] : N[1];
-      for (int n = 1; ok && n < n_max; ++n) {
-        // K of tile n once S(n-1) completed, then V once PV(n-1) completed,
-        // lane A before lane B: the order in which those events happen.
-        for (int x = 0; ok && x < kLanes; ++x) {
-          if (n >= N[x]) continue;
-          if (!mbar_wait(&bar[8 * x + kBarKEmpty], (n - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-          load_kv(x, n, false);
-          k_issued[x] = n + 1;
+      mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
+      // Tile t goes to slot t mod 2 once the tile before it there (t - 2)
+      // was consumed; K and V advance independently.
+      int kt = 0, vt = 0;
+      PollGuard guard;
+      while (kt < N || vt < N) {
+        bool moved = false;
+        if (kt < N && (kt < kStages || mbar_test(&bar[kBarKEmpty + (kt & 1)], ((kt >> 1) - 1) & 1))) {
+          load_kv(kt, false);
+          ++kt;
+          moved = true;
         }
-        for (int x = 0; ok && x < kLanes; ++x) {
-          if (n >= N[x]) continue;
-          if (!mbar_wait(&bar[8 * x + kBarVEmpty], (n - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-          load_kv(x, n, true);
-          v_issued[x] = n + 1;
+        if (vt < N && (vt < kStages || mbar_test(&bar[kBarVEmpty + (vt & 1)], ((vt >> 1) - 1) & 1))) {
+          load_kv(vt, true);
+          ++vt;
+          moved = true;
         }
+        if (moved) {
+          guard.progress();
+          continue;
+        }
+        if (!guard.idle(abort_flag, a.err)) break;
+        // K(t) frees after S(t - 2), V(t) after PV(t - 2): sleep on the older.
+        if (kt < N && (vt >= N || kt <= vt))
+          mbar_sleep(&bar[kBarKEmpty + (kt & 1)], ((kt >> 1) - 1) & 1, kSleepNs);
+        else
+          mbar_sleep(&bar[kBarVEmpty + (vt & 1)], ((vt >> 1) - 1) & 1, kSleepNs);
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
-        for (int x = 0; x < kLanes; ++x) {
-          if (N[x] == 0) continue;
-          mbar_wait_drain(&bar[8 * x + kBarQ], 0);
-          if (k_issued[x]) mbar_wait_drain(&bar[8 * x + kBarKFull], (k_issued[x] - 1) & 1);
-          if (v_issued[x]) mbar_wait_drain(&bar[8 * x + kBarVFull], (v_issued[x] - 1) & 1);
-        }
+        mbar_wait_drain(&bar[kBarQ], 0);
+        for (int t = (kt > kStages ? kt - kStages : 0); t < kt; ++t)
+          mbar_wait_drain(&bar[kBarKFull + (t & 1)], (t >> 1) & 1);
+        for (int t = (vt > kStages ? vt - kStages : 0); t < vt; ++t)
+          mbar_wait_drain(&bar[kBarVFull + (t & 1)], (t >> 1) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -348,108 +403,110 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
-      bool ok = true;
-      for (int x = 0; ok && x < kLanes; ++x) {
-        if (N[x] == 0) continue;
-        uint64_t* b = bar + 8 * x;
-        ok = mbar_wait(&b[kBarQ], 0, abort_flag, a.err) && mbar_wait(&b[kBarKFull], 0, abort_flag, a.err);
-        if (!ok) break;
+      // S(j) into buffer j mod 2, after PV(j - 2) (which read P(j - 2) from
+      // that buffer; tcgen05.mma executes in issue order).
+      auto issue_score = [&](int j) -> bool {
+        if (!mbar_wait(&bar[kBarKFull + (j & 1)], (j >> 1) & 1, abort_flag, a.err)) return false;
         tc_fence_after();
-        issue_s<D>(tmem + 256u * x, q_addr + x * L::kTileBytes, k_addr + x * L::kTileBytes);
-        mma_commit(&b[kBarSFull]);
-        mma_commit(&b[kBarKEmpty]);
-      }
-      int np[kLanes] = {0, 0};
-      while (ok && (np[0] < N[0] || np[1] < N[1])) {
-        for (int x = 0; ok && x < kLanes; ++x) {
-          const int n = np[x];
-          if (n >= N[x]) continue;
-          uint64_t* b = bar + 8 * x;
-          if (!mbar_wait(&b[kBarPFull], n & 1, abort_flag, a.err) ||
-              !mbar_wait(&b[kBarVFull], n & 1, abort_flag, a.err)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv<D>(tmem + 256u * x + kOCol, tmem + 256u * x, v_addr + x * L::kTileBytes, n > 0);
-          mma_commit(&b[kBarVEmpty]);
-          if (n + 1 == N[x]) mma_commit(&b[kBarODone]);  // O final: the epilogue's single wait
-          np[x] = n + 1;
-          if (n + 1 < N[x]) {
-            // S(n+1) overwrites the columns holding P(n); PV(n) was issued
-            // before it by this thread and tcgen05.mma executes in issue
-            // order. Its commit also covers PV(n): once S(n+1) is reported
-            // complete, O holds PV(0..n) and may be rescaled.
-            if (!mbar_wait(&b[kBarKFull], (n + 1) & 1, abort_flag, a.err)) { ok = false; break; }
-            tc_fence_after();
-            issue_s<D>(tmem + 256u * x, q_addr + x * L::kTileBytes, k_addr + x * L::kTileBytes);
-            mma_commit(&b[kBarSFull]);
-            mma_commit(&b[kBarKEmpty]);
-          }
-        }
+        issue_s<D>(tmem + 128u * (j & 1), q_addr, k_addr + (j & 1) * L::kTileBytes);
+        mma_commit(&bar[kBarSFull + (j & 1)]);
+        mma_commit(&bar[kBarKEmpty + (j & 1)]);
+        return true;
+      };
+      bool ok = mbar_wait(&bar[kBarQ], 0, abort_flag, a.err) && issue_score(0);
+      if (ok && N > 1) ok = issue_score(1);
+      for (int i = 0; ok && i < N; ++i) {
+        if (!mbar_wait(&bar[kBarPFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err) ||
+            !mbar_wait(&bar[kBarVFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err))
+          break;
+        tc_fence_after();
+        issue_pv<D>(tmem + kOCol, tmem + 128u * (i & 1), v_addr + (i & 1) * L::kTileBytes, i > 0);
+        mma_commit(&bar[kBarVEmpty + (i & 1)]);
+        mma_commit(&bar[kBarPVDone]);
+        if (i + 1 == N) mma_commit(&bar[kBarODone]);  // O final: the epilogue's wait
+        if (i + 2 < N) ok = issue_score(i + 2);
       }
       mma_commit(&bar[kBarDrain]);
       mbar_wait_drain(&bar[kBarDrain], 0);
     }
-  } else if (warp < kLanes * 4) {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     const Dims& d = a.d;
-    const int x = warp >> 2;           // lane (query tile) of this warp group
-    const int r = tid & 127;           // query row of the tile = TMEM lane
-    const int Nx = N[x];
-    const int Ex = E_of[x];
-    const uint32_t* ents = reinterpret_cast<const uint32_t*>(smem + L::kEnt) + x * kAttnMaxEntries;
-    uint64_t* b = bar + 8 * x;
-    const uint32_t trow = tmem + 256u * x + ((uint32_t)((warp & 3) * 32) << 16);
-    const int qsel = r >> 6;   // warp-uniform
+    const int quarter = warp & 3;        // TMEM lane quarter: rows 32 quarter ..
+    const int half = warp >> 2;          // key columns 64 half .. + 63
+    const int r = quarter * 32 + lane;   // query row of the tile = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int mbit = r >> 6;             // this row's bit in a unit mask (warp-uniform)
+    // red[buf][half][row]: partial row maxima; lsum[half][row]; okf[slot][half][quarter]
+    // (slots 0 and 1 per tile, slot 2 for the epilogue)
+    float* red = reinterpret_cast<float*>(smem + L::kRed);
+    float* lsum = red + 2 * 2 * 128;
+    volatile int* okf = reinterpret_cast<volatile int*>(lsum + 2 * 128);
     const float sc = a.scale_log2;
     float m_used = -INFINITY;  // running maximum in scaled log2 units (possibly stale by < 8)
-    float l_run = 0.f;
-    bool ok = Nx > 0;
-    for (int n = 0; ok && n < Nx; ++n) {
-      ok = mbar_wait(&b[kBarSFull], n & 1, abort_flag, a.err);
-      ok = __all_sync(0xFFFFFFFFu, ok);
+    float l_run = 0.f;         // over this warp's half of the keys
+    bool ok = true;
+    for (int i = 0; i < N; ++i) {
+      const int buf = i & 1;
+      const uint32_t scol = 128u * buf + 64u * half;
+      bool mine = mbar_wait(&bar[kBarSFull + buf], (i >> 1) & 1, abort_flag, a.err);
+      mine = __all_sync(0xFFFFFFFFu, mine);
+      uint32_t s[2][32];
+      float pm = -INFINITY;
+      if (mine) {
+        tc_fence_after();
+        tmem_ld32(trow + scol, s[0]);
+        tmem_ld32(trow + scol + 32u, s[1]);
+        const uint32_t e = ents[2 * i + half];
+        const int lim = ((e >> mbit) & 1u) ? (int)((e >> 8) & 0xFFu) : 0;
+        tmem_wait_ld();
+        if (lim < 64) {  // warp-uniform
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (32 * j + c >= lim) s[j][c] = __float_as_uint(-INFINITY);
+        }
+        float mx[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          mx[j] = fmaxf(__uint_as_float(s[j][0]), __uint_as_float(s[j][1]));
+#pragma unroll
+          for (int c = 2; c < 32; c += 2) mx[j] = max3f(mx[j], __uint_as_float(s[j][c]), __uint_as_float(s[j][c + 1]));
+        }
+        pm = fmaxf(mx[0], mx[1]);
+      }
+      // Both warps of the pair reach this barrier once per tile, whatever
+      // happened: it orders the maxima exchange, guarantees the partner has
+      // read its scores before P overwrites them, and lets both leave together.
+      red[(buf * 2 + half) * 128 + r] = pm;
+      if (lane == 0) okf[(buf * 2 + half) * 4 + quarter] = mine ? 1 : 0;
+      pair_sync(quarter);
+      ok = mine && okf[(buf * 2 + (half ^ 1)) * 4 + quarter] != 0;
       if (!ok) break;
-      tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld32(trow + (uint32_t)(32 * i), s[i]);
-      const uint32_t e0 = ents[2 * n];
-      const uint32_t e1 = (2 * n + 1 < Ex) ? ents[2 * n + 1] : 0u;
-      const int lim0 = ((e0 >> qsel) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
-      const int lim1 = ((e1 >> qsel) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
-      const bool full = (lim0 == 64) && (lim1 == 64);   // warp-uniform
-      tmem_wait_ld();
-      if (!full) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int lim = i < 2 ? lim0 - 32 * i : lim1 - 32 * (i - 2);
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c >= lim) s[i][c] = __float_as_uint(-INFINITY);
-        }
-      }
-      float ma = -INFINITY, mb = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          ma = max3f(ma, __uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1]));
-          mb = max3f(mb, __uint_as_float(s[i][c + 2]), __uint_as_float(s[i][c + 3]));
-        }
-      }
-      const float mt = fmaxf(ma, mb) * sc;  // -inf when nothing is valid
+      const float mt = fmaxf(pm, red[(buf * 2 + (half ^ 1)) * 128 + r]) * sc;  // -inf when nothing is valid
       const bool need = mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt > -INFINITY);
-      if (__any_sync(0xFFFFFFFFu, need)) {
+      if (__any_sync(0xFFFFFFFFu, need)) {  // same rows, same decision in both warps of the pair
         const float m_new = need ? mt : m_used;
         const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
-        if (n > 0) {
-          // O holds PV(0..n-1): the commit of S(n) covered PV(n-1).
+        if (i > 0) {
+          // O must hold PV(0..i-1) before it is scaled. A failed wait skips
+          // the scaling but not the pair's barriers: the abort flag is up and
+          // both warps leave at the next tile's barrier.
+          bool done = mbar_wait(&bar[kBarPVDone], (i - 1) & 1, abort_flag, a.err);
+          done = __all_sync(0xFFFFFFFFu, done);
+          if (done) {
+            tc_fence_after();
 #pragma unroll 1
-          for (int i = 0; i < D / 16; ++i) {
-            uint32_t o[16];
-            tmem_ld16(trow + kOCol + (uint32_t)(16 * i), o);
-            tmem_wait_ld();
+            for (int j = 0; j < D / 32; ++j) {
+              const uint32_t oc = trow + kOCol + (uint32_t)(D / 2) * half + 16u * j;
+              uint32_t o[16];
+              tmem_ld16(oc, o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st16(trow + kOCol + (uint32_t)(16 * i), o);
+              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st16(oc, o);
+            }
           }
         }
         l_run *= alpha;
@@ -460,44 +517,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 nb2 = make_float2(-base, -base);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
+      for (int j = 0; j < 2; ++j) {
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
+          const float2 xv = ffma2(make_float2(__uint_as_float(s[j][2 * q]), __uint_as_float(s[j][2 * q + 1])),
                                   sc2, nb2);
           const float2 p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
           if (q & 1) acc1 = fadd2(acc1, p);
           else acc0 = fadd2(acc0, p);
           pk[q] = cvt_bf16x2(p.x, p.y);
         }
-        tmem_st16(trow + (uint32_t)(16 * h), pk);
+        // bf16 pairs: keys 64 half + 32 j .. go to packed columns 32 half + 16 j
+        tmem_st16(trow + 128u * buf + 32u * half + 16u * j, pk);
       }
       l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&b[kBarPFull]);
+      mbar_arrive(&bar[kBarPFull + buf]);
     }
     // ------------------------------------------------------------ epilogue
+    bool fin = false;
     if (ok) {
-      ok = mbar_wait(&b[kBarODone], 0, abort_flag, a.err);
-      ok = __all_sync(0xFFFFFFFFu, ok);
+      fin = mbar_wait(&bar[kBarODone], 0, abort_flag, a.err);
+      fin = __all_sync(0xFFFFFFFFu, fin);
+      lsum[half * 128 + r] = l_run;
+      if (lane == 0) okf[(2 * 2 + half) * 4 + quarter] = fin ? 1 : 0;
+      pair_sync(quarter);  // both warps of the pair got here: both left the loop with ok
+      fin = fin && okf[(2 * 2 + (half ^ 1)) * 4 + quarter] != 0;
     }
-    if (ok) {
+    if (fin) {
       tc_fence_after();
-      const int pr = m_of[x] * kBM + r;  // row in the padded chunk
+      const float l_tot = l_run + lsum[(half ^ 1) * 128 + r];
+      const int pr = m * kBM + r;  // row in the padded chunk
       const int f = pr / d.T_pad;
       const int rr = pr - f * d.T_pad;
       const bool row_ok = (f < d.Fc) && (rr < d.T_f);
       const int bb = bh / d.H;
       const int h = bh - bb * d.H;
       const size_t n_tok = (size_t)f * d.T_f + rr;
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      uint16_t* orow = a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D;
+      const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      uint16_t* orow = a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D + (D / 2) * half;
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
+      for (int i = 0; i < D / 64; ++i) {
         uint32_t o[32];
-        tmem_ld32(trow + kOCol + (uint32_t)(32 * i), o);
+        tmem_ld32(trow + kOCol + (uint32_t)(D / 2) * half + 32u * i, o);
         tmem_wait_ld();
         if (row_ok) {
           uint32_t pk[16];
@@ -510,8 +574,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (row_ok && a.lse)
-        a.lse[(size_t)bh * d.Lq + n_tok] = (m_used + log2f(l_run)) * 0.69314718055994531f;
+      if (row_ok && half == 0 && a.lse)
+        a.lse[(size_t)bh * d.Lq + n_tok] = (m_used + log2f(l_tot)) * 0.69314718055994531f;
     }
   }
 
@@ -561,7 +625,7 @@ static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.MT + kLanes - 1) / kLanes, a.d.B * a.d.H);
+  dim3 grid(a.MT, a.d.B * a.d.H);
   attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }

@@ -81,12 +81,20 @@ __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy (TMA, tensor core) accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -96,6 +104,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking probe of a phase (for roles that serve several barriers).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspends the thread until the phase completes or about `ns` nanoseconds
+// passed (a polling role's idle step: a suspended thread takes no issue
+// slots from the warps that share its scheduler).
+__device__ __forceinline__ bool mbar_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
@@ -121,6 +157,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
 }
+
+// Bounded polling loop of a role that serves several barriers: `idle()` is
+// called after a round that made no progress and returns false (after
+// latching CVA_DEV_TIMEOUT and raising the abort flag) once no progress was
+// made for `kWaitLimitNs`, or when another role raised the flag.
+struct PollGuard {
+  uint64_t t_last = 0;
+  uint32_t it = 0;
+  __device__ __forceinline__ void progress() { it = 0; }
+  __device__ __forceinline__ bool idle(volatile int* abort_flag, int* err) {
+    if (it == 0) t_last = globaltimer_ns();
+    if ((++it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t_last > kWaitLimitNs) {
+        *abort_flag = 1;
+        latch_error(err, CVA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+    return true;
+  }
+};
 
 // 3D tiled TMA load global -> shared, completion counted on `bar` (bytes).
 // No multicast: every CTA fetches its own tiles.

@@ -67,7 +67,7 @@ struct AttnArgs {
   int MT;                    // 128-row query tiles per (b, h)
   float scale_log2;          // log2(e) / sqrt(D)
 };
-constexpr int kAttnMaxEntries = 2048;     // 64-row key units per CTA
+constexpr int kAttnMaxEntries = 4096;     // 64-row key units per CTA (two query tiles)
 constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
 
 // Builds the tensor maps and launches the attention kernel.
