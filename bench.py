@@ -47,6 +47,12 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="chunks 1..N of the workload under its literal and mirrored density "
+                         "schedules, one JSON line each (measurement mode, not the bench line)")
+    ap.add_argument("--stream", action="store_true",
+                    help="streaming run: every chunk of the workload through all its layers, "
+                         "per-chunk latency percentiles (measurement mode, not the bench line)")
     return ap.parse_args()
 
 
@@ -77,16 +83,17 @@ def host_cores():
 
 # ---------------------------------------------------------------- workloads
 
-def setup_workload(args, layer):
+def setup_workload(args, layer, wl=None):
     """Device state of one chunk: tables, cache with history, inputs, budget."""
     import numpy as np
     import torch
     from autoregressive_video_dit_b200 import ops
     from cva_workload import WORKLOADS, chunk_inputs, key_centres
 
-    wl = WORKLOADS[args.workload]
-    if args.chunk is not None:
-        wl = wl.with_chunk(args.chunk)
+    if wl is None:
+        wl = WORKLOADS[args.workload]
+        if args.chunk is not None:
+            wl = wl.with_chunk(args.chunk)
     shape = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
     tables = ops.DeviceRopeTables(wl.D, wl.t0 + wl.Fc, wl.Fh, wl.Fw)
     cache = ops.DeviceKVCache(shape, wl.window, 0)
@@ -286,6 +293,57 @@ class OracleSample:
         return flops / dt / 1e12, desc, dt, flops
 
 
+# ---------------------------------------------------------------- timing
+
+def time_steps(step, flush, n, stream):
+    """Runs `step` n times, L2 flushed before each, with the library's stage
+    events (start, after rotate/append/pool, after selection, after
+    attention) recorded on `stream`. Returns per-step lists in ms: whole
+    step, rotate/append/pool, selection, attention."""
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for evs in st_ev:
+        for e in evs:
+            e.record(stream)           # create the underlying events
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush.zero_()
+        ops.set_stage_events(st_ev[i])
+        step()
+    ops.set_stage_events(None)
+    torch.cuda.synchronize()
+    return ([e[0].elapsed_time(e[3]) for e in st_ev], [e[0].elapsed_time(e[1]) for e in st_ev],
+            [e[1].elapsed_time(e[2]) for e in st_ev], [e[2].elapsed_time(e[3]) for e in st_ev])
+
+
+def reduce_over_ranks(ms, work, device):
+    """Weak scaling over independent instances: the job takes as long as its
+    slowest rank (max of `ms`) and does the sum of the ranks' `work`. With
+    no process group, or one rank, the values pass through."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), float(work)
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([float(work)], device=device, dtype=torch.float64)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(w.item())
+
+
+def rank_layer(rank):
+    """Each rank runs its own instance on the inputs of its own layer seed."""
+    return rank
+
+
+def percentile(xs, q):
+    """Nearest-rank percentile (q in [0, 100]) of a non-empty list."""
+    ys = sorted(xs)
+    k = max(1, math.ceil(q / 100.0 * len(ys)))
+    return ys[k - 1]
+
+
 # ---------------------------------------------------------------- main arms
 
 def run_reference(args):
@@ -339,7 +397,7 @@ def run_cuda(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     from autoregressive_video_dit_b200 import ops
 
-    st = setup_workload(args, layer=rank)
+    st = setup_workload(args, layer=rank_layer(rank))
     wl = st["wl"]
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -355,43 +413,19 @@ def run_cuda(args):
     assert ops.device_status() == 0
     flops = attention_flops(st)
 
-    # stage events: start, after rotate/append/pool, after selection, after attention
     n = args.steps
-    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
-    for evs in st_ev:
-        for e in evs:
-            e.record(stream)           # create the underlying events
-    torch.cuda.synchronize()
     sampler = ClockSampler(enabled=not args.no_clocks)
     time.sleep(0.3 if not args.no_clocks else 0)
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(n):
-        flush.zero_()
-        ops.set_stage_events(st_ev[i])
-        step()
-    ops.set_stage_events(None)
-    torch.cuda.synchronize()
+    step_ms, rope_ms, sel_ms, attn_ms = time_steps(step, flush, n, stream)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     assert ops.device_status() == 0
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in st_ev]
-    rope_ms = [e[0].elapsed_time(e[1]) for e in st_ev]
-    sel_ms = [e[1].elapsed_time(e[2]) for e in st_ev]
-    attn_ms = [e[2].elapsed_time(e[3]) for e in st_ev]
     ms = statistics.mean(step_ms)
-    ms_max = ms
-    total_flops = flops
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        fsum = torch.tensor([flops], device="cuda", dtype=torch.float64)
-        dist.all_reduce(fsum, op=dist.ReduceOp.SUM)
-        total_flops = float(fsum.item())
+    ms_max, total_flops = reduce_over_ranks(ms, flops, "cuda")
 
     # end to end through the public call with pinned host buffers
     e2e = None
@@ -414,11 +448,7 @@ def run_cuda(args):
             if i >= 2:
                 evs[i - 2][1].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms, _ = reduce_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), 0.0, "cuda")
         nbytes = lambda t: t.numel() * t.element_size()
         e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": nbytes(hq) + nbytes(hk) + nbytes(hv),
@@ -481,10 +511,117 @@ def run_cuda(args):
     return 0
 
 
+def run_sweep(args):
+    """Per-chunk cost under the density schedule and its mirror (chunk 1 is
+    dense: no history)."""
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    from cva_workload import WORKLOADS
+    base = WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for sched, slope in (("literal", base.d_slope), ("mirrored", -base.d_slope)):
+        for chunk in range(1, base.chunks + 1):
+            wl = base.replace(d_slope=slope).with_chunk(chunk)
+            st = setup_workload(args, layer=0, wl=wl)
+
+            def step():
+                ops.chunk_attention(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0,
+                                    st["k_f"], st["k_b"], st["ws"], st["out"])
+
+            for _ in range(max(args.warmup, 1)):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
+            assert ops.device_status() == 0
+            flops = attention_flops(st)
+            step_ms, rope_ms, sel_ms, attn_ms = time_steps(step, flush, args.steps, stream)
+            assert ops.device_status() == 0
+            ms = statistics.median(step_ms)
+            print(json.dumps({
+                "mode": "schedule sweep", "workload": wl.key, "schedule": sched, "chunk": chunk,
+                "history_frames": st["F"], "k_f": st["k_f"], "k_b": st["k_b"],
+                "ms": ms, "attention_ms": statistics.median(attn_ms),
+                "select_us": 1e3 * statistics.median(sel_ms),
+                "select_share": statistics.median(sel_ms) / ms,
+                "rotate_append_pool_us": 1e3 * statistics.median(rope_ms),
+                "attention_tflop": flops / 1e12,
+                "attention_tflops": flops / (statistics.median(attn_ms) * 1e-3) / 1e12,
+                "steps": args.steps, "stat": "median"}), flush=True)
+            del st
+    return 0
+
+
+def run_stream(args):
+    """Every chunk of the workload once, through all its layers, each layer
+    with its own cache (rolling window); per-chunk latency = the sum over
+    layers, timed from the first layer's start to the last layer's end.
+    Inputs are drawn on the device from a seeded generator per (chunk,
+    layer), outside the timed region."""
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    from cva_workload import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    shape = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
+    tables = ops.DeviceRopeTables(wl.D, wl.Fc * wl.chunks, wl.Fh, wl.Fw)
+    caches = [ops.DeviceKVCache(shape, wl.window, 0) for _ in range(wl.layers)]
+    budgets = []
+    for c in range(1, wl.chunks + 1):
+        hist = min(wl.Fc * (c - 1), wl.window - wl.Fc)
+        budgets.append(ops.cag_budget(c, hist, wl.nb, dense=wl.dense, k_f_max=wl.k_f_max,
+                                      d_base=(wl.d_base.numerator, wl.d_base.denominator),
+                                      d_slope=(wl.d_slope.numerator, wl.d_slope.denominator),
+                                      pivot=wl.d_pivot, k_b_fixed=wl.k_b_fixed) if hist > 0 else (0, 0))
+    k_f_max = max(b[0] for b in budgets)
+    k_b_max = max(b[1] for b in budgets)
+    ws = torch.empty(ops.chunk_workspace_bytes(shape, k_f_max, k_b_max), dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    gen = torch.Generator(device="cuda")
+    size = (wl.B, wl.Lq, wl.H, wl.D)
+
+    def inputs(c, layer):
+        gen.manual_seed(1_000_000 * wl.config_index + 1_000 * c + layer)
+        return [torch.randn(size, generator=gen, device="cuda").to(torch.bfloat16) for _ in range(3)]
+
+    def run_chunk(c, timed):
+        k_f, k_b = budgets[c - 1]
+        t0 = wl.t0_of(c)
+        xs = [inputs(c, layer) for layer in range(wl.layers)]
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for layer in range(wl.layers):
+            q, k, v = xs[layer]
+            ops.chunk_attention(q, k, v, caches[layer], tables, t0, k_f, k_b, ws, out)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) if timed else None
+
+    for c in (1, 2):                      # warm-up, then the caches start over
+        run_chunk(c, False)
+    caches = [ops.DeviceKVCache(shape, wl.window, 0, arena=x.arena) for x in caches]
+    lat = [run_chunk(c, True) for c in range(1, wl.chunks + 1)]
+    assert ops.device_status() == 0
+    full = wl.window // wl.Fc + 1          # first chunk whose history fills the window
+    steady = lat[full - 1:]
+    print(json.dumps({
+        "mode": "streaming", "workload": wl.key, "chunks": wl.chunks, "layers": wl.layers,
+        "window_frames": wl.window, "unit": "ms per chunk (all layers)",
+        "p50": percentile(lat, 50), "p99": percentile(lat, 99), "max": max(lat),
+        "chunk1": lat[0], "steady_p50": percentile(steady, 50), "steady_from_chunk": full,
+        "budget_first_full_window": {"k_f": budgets[full - 1][0], "k_b": budgets[full - 1][1]},
+        "per_chunk": [round(x, 3) for x in lat]}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
+    if args.stream:
+        return run_stream(args)
     return run_cuda(args)
 
 
