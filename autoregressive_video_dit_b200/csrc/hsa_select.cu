@@ -3,21 +3,24 @@
 // history frames are picked with frame-pooled keys, then the important
 // blocks inside those frames with block-pooled keys.
 //
-// One warp per (batch*head, query block). Scores are dot products of the
-// block-pooled query with pooled keys, 32 at a time: each lane forms the
-// partial dot products of its D/32 slice for 32 candidates, and a
-// reduce-scatter through warp shuffles (31 exchanges) leaves candidate
-// base+i's score on lane i. Every candidate becomes a 64-bit key (order-
-// preserving score bits, then the complement of its position) so that a
-// descending sort ranks by score and breaks ties toward the lower
-// position. The warp sorts its keys with a bitonic network in its own
-// slice of shared memory; the k-th key is the threshold, and the chosen
-// positions are emitted in ascending order with ballots.
+// One CTA of 256 threads per (batch*head, query block). Scores are dot
+// products of the block-pooled query with pooled keys, 32 at a time per
+// warp: each lane forms the partial dot products of its D/32 slice for 32
+// candidates, and a reduce-scatter through warp shuffles (31 exchanges)
+// leaves candidate base+i's score on lane i; the warps share the candidate
+// groups. Every candidate becomes a 64-bit key (order-preserving score bits,
+// then the complement of its position), so keys are distinct and "ranks by
+// score, ties toward the lower position" is their descending order. A
+// candidate's rank is the number of keys above it (each thread counts over
+// the keys in shared memory); it is picked when its rank is below k. The
+// picked positions are written in ascending order by a CTA-wide ordered
+// compaction (warp ballots plus a scan of the per-warp counts).
 #include "kernels.cuh"
 
 namespace cva {
 
-constexpr int kSelWarps = 4;
+constexpr int kSelThreads = 256;
+constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelMaxFrames = 256;
 
 __device__ __forceinline__ uint32_t ordered_bits(float s) {
@@ -28,38 +31,19 @@ __device__ __forceinline__ uint64_t rank_key(float s, int pos) {
   return ((uint64_t)ordered_bits(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)pos);
 }
 
-// Descending bitonic sort of key[0..N) (N a power of two) by one warp.
-__device__ void warp_bitonic_desc(uint64_t* key, int N) {
-  const int lane = threadIdx.x & 31;
-  for (int k = 2; k <= N; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int p = lane; p < (N >> 1); p += 32) {
-        const int i = 2 * p - (p & (j - 1));  // the member of the pair with bit j clear
-        const int l = i + j;
-        const uint64_t x = key[i], y = key[l];
-        const bool desc = (i & k) == 0;
-        if (desc ? (x < y) : (x > y)) {
-          key[i] = y;
-          key[l] = x;
-        }
-      }
-      __syncwarp();
-    }
-  }
-}
-
 // Scores of candidates base .. base+31 (those below `count`); lane i returns
-// candidate base+i's score. `row_of(c)` gives candidate c's pooled key row.
-template <int D, class RowOf>
+// candidate base+i's score. Candidate c's pooled key row starts at
+// rows + rowoff[c] (floats; rowoff in shared memory).
+template <int D>
 __device__ __forceinline__ float score_group(const float (&q)[D / 32], int base, int count,
-                                             RowOf row_of) {
+                                             const float* rows, const int* rowoff) {
   const int lane = threadIdx.x & 31;
   float v[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     float s = 0.f;
     if (base + c < count) {
-      const float* p = row_of(base + c) + lane * (D / 32);
+      const float* p = rows + rowoff[base + c] + lane * (D / 32);
       if constexpr (D == 128) {
         const float4 kv = *reinterpret_cast<const float4*>(p);
         s = q[0] * kv.x + q[1] * kv.y + q[2] * kv.z + q[3] * kv.w;
@@ -83,27 +67,62 @@ __device__ __forceinline__ float score_group(const float (&q)[D / 32], int base,
   return v[0];
 }
 
-__host__ __device__ inline int pow2_at_least(int n) {
-  int p = 32;
-  while (p < n) p <<= 1;
-  return p;
+// Number of keys in key[0..n) above key[i]; key[] is padded with zeros
+// (below every real key) to an even length. Two keys per shared-memory
+// read, the same address across the warp (a broadcast).
+__device__ __forceinline__ int rank_of(const uint64_t* key, int n, int i) {
+  const uint64_t x = key[i];
+  const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(key);
+  int r = 0;
+  for (int j = 0; j < (n + 1) >> 1; ++j) {
+    const ulonglong2 y = k2[j];
+    r += (y.x > x ? 1 : 0) + (y.y > x ? 1 : 0);
+  }
+  return r;
+}
+
+// Ordered compaction over positions 0..n-1: `emit(slot, pos)` for every pos
+// with take(pos), slots counted in ascending pos. Returns the number taken.
+// All threads of the CTA call it.
+template <class Take, class Emit>
+__device__ int compact(int n, int* warp_cnt, Take take, Emit emit) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int base = 0;
+  for (int c0 = 0; c0 < n; c0 += kSelThreads) {
+    const int c = c0 + tid;
+    const bool t = c < n && take(c);
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, t);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+      const int cw = warp_cnt[w];
+      before += w < warp ? cw : 0;
+      total += cw;
+    }
+    if (t) emit(base + before + __popc(bal & ((1u << lane) - 1u)), c);
+    base += total;
+    __syncthreads();
+  }
+  return base;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSelWarps * 32) hsa_select_kernel(SelectArgs a, int nmax) {
+__global__ void __launch_bounds__(kSelThreads) hsa_select_kernel(SelectArgs a, int nmax) {
   extern __shared__ uint8_t sel_smem[];
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  __shared__ int warp_cnt[kSelWarps];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   const Dims& d = a.d;
-  const int u = blockIdx.x * kSelWarps + warp;
-  if (u >= d.B * d.H * d.NQB) return;
+  const int u = blockIdx.x;
   const int bh = u / d.NQB;
 
-  // per-warp smem: keys[nmax] u64, score[nmax] f32, chosen frames[256] i32
-  uint8_t* base_ptr = sel_smem + (size_t)warp * ((size_t)nmax * 12 + kSelMaxFrames * 4);
-  uint64_t* key = reinterpret_cast<uint64_t*>(base_ptr);
-  float* score = reinterpret_cast<float*>(base_ptr + (size_t)nmax * 8);
-  int* chosen = reinterpret_cast<int*>(base_ptr + (size_t)nmax * 12);
+  // smem: keys[nmax + 1] u64, chosen frames [256] i32, row offsets [nmax] i32
+  uint64_t* key = reinterpret_cast<uint64_t*>(sel_smem);
+  int* chosen = reinterpret_cast<int*>(sel_smem + (size_t)(nmax + 1) * 8);
+  int* rowoff = chosen + kSelMaxFrames;
 
   float q[D / 32];
   {
@@ -117,88 +136,64 @@ __global__ void __launch_bounds__(kSelWarps * 32) hsa_select_kernel(SelectArgs a
   // ---- level 1: frames ---------------------------------------------------
   const int F = a.F;
   const int kfe = a.k_f < F ? a.k_f : F;
-  const int NF = pow2_at_least(F);
-  auto frame_row = [&](int p) { return kfrm + (size_t)((a.t_lo + p) % a.W) * D; };
-  for (int b0 = 0; b0 < F; b0 += 32) {
-    const float s = score_group<D>(q, b0, F, frame_row);
+  for (int p = tid; p < F; p += kSelThreads) rowoff[p] = ((a.t_lo + p) % a.W) * D;
+  if (tid == 0) key[F] = 0ull;  // pad to an even count
+  __syncthreads();
+  for (int b0 = 32 * warp; b0 < F; b0 += 32 * kSelWarps) {
+    const float s = score_group<D>(q, b0, F, kfrm, rowoff);
     const int p = b0 + lane;
-    if (p < F) score[p] = s;
+    if (p < F) key[p] = rank_key(s, p);
   }
-  __syncwarp();
-  uint64_t thr = 1;  // every real key is above 1
-  if (F > kfe) {
-    for (int p = lane; p < NF; p += 32) key[p] = p < F ? rank_key(score[p], p) : 0ull;
-    __syncwarp();
-    warp_bitonic_desc(key, NF);
-    thr = kfe > 0 ? key[kfe - 1] : ~0ull;
-  }
-  int nsel = 0;
-  for (int b0 = 0; b0 < F; b0 += 32) {
-    const int p = b0 + lane;
-    const bool take = p < F && rank_key(score[p], p) >= thr;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
-    if (take) chosen[nsel + __popc(bal & ((1u << lane) - 1u))] = p;
-    nsel += __popc(bal);
-  }
-  __syncwarp();
+  __syncthreads();
+  const int nsel = compact(
+      F, warp_cnt, [&](int p) { return F <= kfe || rank_of(key, F, p) < kfe; },
+      [&](int slot, int p) { chosen[slot] = p; });
   if (a.frame_idx) {
-    for (int i = lane; i < nsel; i += 32) a.frame_idx[(size_t)u * a.k_f_stride + i] = a.t_lo + chosen[i];
+    for (int i = tid; i < nsel; i += kSelThreads) a.frame_idx[(size_t)u * a.k_f_stride + i] = a.t_lo + chosen[i];
   }
+  // chosen[] is complete: compact() ends with a barrier
 
   // ---- level 2: blocks of the chosen frames --------------------------------
   const int C = nsel * d.nb;
   const int kb = a.k_b;
-  const int NC = pow2_at_least(C);
-  auto cand_row = [&](int c) {
+  for (int c = tid; c < C; c += kSelThreads) {
     const int fi = c / d.nb;
     const int jj = c - fi * d.nb;
-    return kblk + ((size_t)((a.t_lo + chosen[fi]) % a.W) * d.nb + jj) * D;
-  };
-  for (int b0 = 0; b0 < C; b0 += 32) {
-    const float s = score_group<D>(q, b0, C, cand_row);
+    rowoff[c] = (((a.t_lo + chosen[fi]) % a.W) * d.nb + jj) * D;
+  }
+  if (tid == 0) key[C] = 0ull;
+  __syncthreads();
+  for (int b0 = 32 * warp; b0 < C; b0 += 32 * kSelWarps) {
+    const float s = score_group<D>(q, b0, C, kblk, rowoff);
     const int c = b0 + lane;
-    if (c < C) score[c] = s;
+    if (c < C) key[c] = rank_key(s, c);
   }
-  __syncwarp();
-  thr = 1;
-  if (C > kb) {
-    for (int c = lane; c < NC; c += 32) key[c] = c < C ? rank_key(score[c], c) : 0ull;
-    __syncwarp();
-    warp_bitonic_desc(key, NC);
-    thr = kb > 0 ? key[kb - 1] : ~0ull;
-  }
-  int nout = 0;
+  __syncthreads();
   int32_t* out = a.block_idx + (size_t)u * a.k_b_max;
-  for (int b0 = 0; b0 < C; b0 += 32) {
-    const int c = b0 + lane;
-    const bool take = c < C && rank_key(score[c], c) >= thr;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
-    if (take) {
-      const int fi = c / d.nb;
-      out[nout + __popc(bal & ((1u << lane) - 1u))] = (a.t_lo + chosen[fi]) * d.nb + (c - fi * d.nb);
-    }
-    nout += __popc(bal);
-  }
-  if (lane == 0 && a.block_cnt) a.block_cnt[u] = nout;
+  const int nout = compact(
+      C, warp_cnt, [&](int c) { return C <= kb || rank_of(key, C, c) < kb; },
+      [&](int slot, int c) {
+        const int fi = c / d.nb;
+        out[slot] = (a.t_lo + chosen[fi]) * d.nb + (c - fi * d.nb);
+      });
+  if (tid == 0 && a.block_cnt) a.block_cnt[u] = nout;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   const int kfe = a.k_f < a.F ? a.k_f : a.F;
-  const int nf = pow2_at_least(a.F);
-  const int nc = pow2_at_least(kfe * a.d.nb);
-  const int nmax = nf > nc ? nf : nc;
-  const size_t smem = (size_t)kSelWarps * ((size_t)nmax * 12 + kSelMaxFrames * 4);
+  const int nmax = a.F > kfe * a.d.nb ? a.F : kfe * a.d.nb;
+  const size_t smem = (size_t)(nmax + 1) * 8 + kSelMaxFrames * 4 + (size_t)nmax * 4;
   const int units = a.d.B * a.d.H * a.d.NQB;
-  dim3 grid((units + kSelWarps - 1) / kSelWarps);
+  dim3 grid(units);
   cudaError_t e;
   if (a.d.D == 128) {
     e = cudaFuncSetAttribute(hsa_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    hsa_select_kernel<128><<<grid, kSelWarps * 32, smem, stream>>>(a, nmax);
+    hsa_select_kernel<128><<<grid, kSelThreads, smem, stream>>>(a, nmax);
   } else {
     e = cudaFuncSetAttribute(hsa_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    hsa_select_kernel<64><<<grid, kSelWarps * 32, smem, stream>>>(a, nmax);
+    hsa_select_kernel<64><<<grid, kSelThreads, smem, stream>>>(a, nmax);
   }
   return cudaGetLastError();
 }
