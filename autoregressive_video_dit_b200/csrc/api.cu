@@ -124,8 +124,13 @@ void history(const cva_kv_cache* c, int t0, int* t_lo, int* F) {
 }
 
 struct ChunkWs {
-  size_t q_rot, qpool, frame_idx, block_idx, block_cnt, total;
+  size_t q_rot, qpool, frame_idx, block_idx, block_cnt, attn, total;
 };
+
+// Attention scratch: partial (O, max, sum) of the pieces of split tail tiles.
+size_t attn_split_bytes(const Dims& d) {
+  return round256((size_t)kAttnMaxPieces * 128 * d.D * 4) + round256((size_t)kAttnMaxPieces * 128 * 2 * 4);
+}
 
 ChunkWs chunk_ws_layout(const Dims& d, int k_f, int k_b) {
   ChunkWs w;
@@ -136,6 +141,7 @@ ChunkWs chunk_ws_layout(const Dims& d, int k_f, int k_b) {
   w.frame_idx = off; off += round256(bhq * (size_t)(k_f > 0 ? k_f : 0) * 4);
   w.block_idx = off; off += round256(bhq * (size_t)(k_b > 0 ? k_b : 0) * 4);
   w.block_cnt = off; off += round256(bhq * 4);
+  w.attn = off; off += attn_split_bytes(d);
   w.total = off;
   return w;
 }
@@ -460,12 +466,25 @@ int cva_attn_workspace_bytes(const cva_shape* shape, int32_t k_b_max, size_t* by
   if (rc) return rc;
   if (!bytes) return fail(CVA_EINVAL, "bytes is NULL");
   (void)k_b_max;
-  *bytes = 0;
+  *bytes = attn_split_bytes(make_dims(*shape));
   return CVA_OK;
 }
 
+// SMs of the current device (cached per device).
+static int sm_count() {
+  static int counts[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const int32_t* block_idx,
-                     const int32_t* block_cnt, int k_b_max, void* out, float* lse, cudaStream_t s) {
+                     const int32_t* block_cnt, int k_b_max, void* out, float* lse, void* split_ws,
+                     size_t split_bytes, cudaStream_t s) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -485,6 +504,24 @@ static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const
   a.F = F;
   a.MT = (d.Fc * d.T_pad + 127) / 128;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d.D));
+  // Tail split: the tiles of the last, partial wave are cut into key-range
+  // pieces so that they fill the SMs (needs the scratch; else unsplit).
+  const int tiles = a.MT * d.B * d.H;
+  a.Qf = tiles;
+  a.pieces = 1;
+  const int nsm = sm_count();
+  if (split_ws && split_bytes >= attn_split_bytes(d) && nsm > 0) {
+    const int tail = tiles % nsm;
+    int pieces = tail > 0 ? nsm / tail : 0;
+    if (tail > 0 && pieces > kAttnMaxPieces / tail) pieces = kAttnMaxPieces / tail;
+    if (pieces >= 2) {
+      a.Qf = tiles - tail;
+      a.pieces = pieces;
+      a.part_o = static_cast<float*>(split_ws);
+      a.part_ml = reinterpret_cast<float*>(static_cast<char*>(split_ws) +
+                                           round256((size_t)kAttnMaxPieces * 128 * d.D * 4));
+    }
+  }
   const char* why = "";
   cudaError_t e = launch_attention(a, q_rot, cache->k, cache->v, s, &why);
   if (e == cudaErrorInvalidValue && why[0]) return fail(CVA_ELAUNCH, "attention: %s", why);
@@ -495,16 +532,15 @@ int cva_blocksparse_attn_fwd(const void* q_rot, const cva_kv_cache* cache, int32
                              const int32_t* block_idx, const int32_t* block_cnt, int32_t k_b_max,
                              void* out, float* lse, void* workspace, size_t ws_bytes,
                              cva_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!q_rot || !out) return fail(CVA_EINVAL, "q_rot or out is NULL");
   if (!aligned(q_rot, 16) || !aligned(out, 16)) return fail(CVA_EINVAL, "q_rot and out must be 16-byte aligned");
   if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
   if (block_idx && (!block_cnt || k_b_max < 0)) return fail(CVA_EINVAL, "sparse call needs block_cnt and k_b_max >= 0");
+  if (workspace && !aligned(workspace, 256)) return fail(CVA_EINVAL, "workspace must be 256-byte aligned");
   return attn_impl(q_rot, cache, t0, block_idx, block_cnt, block_idx ? k_b_max : 0, out, lse,
-                   static_cast<cudaStream_t>(stream));
+                   workspace, workspace ? ws_bytes : 0, static_cast<cudaStream_t>(stream));
 }
 
 int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, size_t* bytes) {
@@ -584,7 +620,7 @@ int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_k
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   // step 5
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, s);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;

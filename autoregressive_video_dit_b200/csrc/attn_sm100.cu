@@ -36,6 +36,12 @@
 // Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
 // roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait and the tensor memory is released.
+//
+// Tail split: the tiles of the last, partial wave of CTAs would leave most
+// SMs idle for a whole tile's time. Given scratch, the host cuts each of
+// them into `pieces` contiguous ranges of its key tiles; a piece writes its
+// unnormalised O, running maximum and sum, and attn_merge_kernel combines
+// the pieces of a tile (flash-decoding style) into bf16 O and LSE.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -298,8 +304,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int bh = blockIdx.y;
-  const int m = blockIdx.x;  // query tile
+  // Work item: a whole tile, or one key-range piece of a tail tile.
+  int tile = blockIdx.x, piece = 0, slot = -1;
+  if (tile >= a.Qf) {
+    const int k = tile - a.Qf;
+    tile = a.Qf + k / a.pieces;
+    piece = k % a.pieces;
+    slot = k;                  // partial-result slot
+  }
+  const int bh = tile / a.MT;
+  const int m = tile - bh * a.MT;  // query tile
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -331,7 +345,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const Stream st = build_stream(a, m, false, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
                                  reinterpret_cast<uint32_t*>(smem + L::kCnt), tot);
-  const int N = st.total();  // key tiles, in stream order
+  const int NT = st.total();  // key tiles of the tile, in stream order
+  // This work item's key tiles: all, or piece `piece` of `pieces`.
+  const int i_lo = slot < 0 ? 0 : (int)((int64_t)NT * piece / a.pieces);
+  const int N = slot < 0 ? NT : (int)((int64_t)NT * (piece + 1) / a.pieces) - i_lo;
+  const uint32_t* units = ents + 2 * i_lo;  // units of local key tile i: units[2i], units[2i+1]
   // the build scratch in the V ring is dead; the async proxy may now write it
   fence_proxy_async_smem();
   tc_fence_before();
@@ -346,7 +364,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       auto load_kv = [&](int t, bool is_v) {
-        const uint32_t e0 = ents[2 * t], e1 = ents[2 * t + 1];
+        const uint32_t e0 = units[2 * t], e1 = units[2 * t + 1];
         const int r0 = (int)(e0 >> 16) * 64;
         const int r1 = (int)(e1 >> 16) * 64;
         const int s = t & 1;
@@ -359,9 +377,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_3d(dst + c * L::kChunkBytes + 8192, map, full, c * 64, r1, bh);
         }
       };
-      mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
+      if (N > 0) {
+        mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
+      }
       // Tile t goes to slot t mod 2 once the tile before it there (t - 2)
       // was consumed; K and V advance independently.
       int kt = 0, vt = 0;
@@ -390,7 +410,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_sleep(&bar[kBarVEmpty + (vt & 1)], ((vt >> 1) - 1) & 1, kSleepNs);
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
-        mbar_wait_drain(&bar[kBarQ], 0);
+        if (N > 0) mbar_wait_drain(&bar[kBarQ], 0);
         for (int t = (kt > kStages ? kt - kStages : 0); t < kt; ++t)
           mbar_wait_drain(&bar[kBarKFull + (t & 1)], (t >> 1) & 1);
         for (int t = (vt > kStages ? vt - kStages : 0); t < vt; ++t)
@@ -413,7 +433,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mma_commit(&bar[kBarKEmpty + (j & 1)]);
         return true;
       };
-      bool ok = mbar_wait(&bar[kBarQ], 0, abort_flag, a.err) && issue_score(0);
+      bool ok = N > 0 && mbar_wait(&bar[kBarQ], 0, abort_flag, a.err) && issue_score(0);
       if (ok && N > 1) ok = issue_score(1);
       for (int i = 0; ok && i < N; ++i) {
         if (!mbar_wait(&bar[kBarPFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err) ||
@@ -457,7 +477,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         tmem_ld32(trow + scol, s[0]);
         tmem_ld32(trow + scol + 32u, s[1]);
-        const uint32_t e = ents[2 * i + half];
+        const uint32_t e = units[2 * i + half];
         const int lim = ((e >> mbit) & 1u) ? (int)((e >> 8) & 0xFFu) : 0;
         tmem_wait_ld();
         if (lim < 64) {  // warp-uniform
@@ -539,14 +559,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ epilogue
     bool fin = false;
     if (ok) {
-      fin = mbar_wait(&bar[kBarODone], 0, abort_flag, a.err);
+      fin = N == 0 || mbar_wait(&bar[kBarODone], 0, abort_flag, a.err);  // an empty piece has no PV
       fin = __all_sync(0xFFFFFFFFu, fin);
       lsum[half * 128 + r] = l_run;
       if (lane == 0) okf[(2 * 2 + half) * 4 + quarter] = fin ? 1 : 0;
       pair_sync(quarter);  // both warps of the pair got here: both left the loop with ok
       fin = fin && okf[(2 * 2 + (half ^ 1)) * 4 + quarter] != 0;
     }
-    if (fin) {
+    if (fin && slot >= 0) {
+      // A piece of a split tile: raw O (relative to the running maximum),
+      // the maximum and the sum, for the merge launch.
+      if (N > 0) tc_fence_after();
+      const float l_tot = l_run + lsum[(half ^ 1) * 128 + r];
+      float* po = a.part_o + ((size_t)slot * kBM + r) * D + (D / 2) * half;
+#pragma unroll
+      for (int i = 0; i < D / 64; ++i) {
+        uint32_t o[32];
+        if (N > 0) {
+          tmem_ld32(trow + kOCol + (uint32_t)(D / 2) * half + 32u * i, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        float4* dst = reinterpret_cast<float4*>(po + 32 * i);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                               __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+      }
+      if (half == 0)
+        reinterpret_cast<float2*>(a.part_ml)[(size_t)slot * kBM + r] = make_float2(m_used, l_tot);
+    } else if (fin) {
       tc_fence_after();
       const float l_tot = l_run + lsum[(half ^ 1) * 128 + r];
       const int pr = m * kBM + r;  // row in the padded chunk
@@ -587,6 +631,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
+// Combines the pieces of the split tail tiles: per row, the maximum M of
+// the pieces' running maxima, sum = sum_p l_p 2^(m_p - M), o = sum_p o_p
+// 2^(m_p - M) / sum. One CTA per row of a split tile, D/4 threads (four
+// columns each).
+template <int D>
+__global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a) {
+  const Dims& d = a.d;
+  const int tt = blockIdx.x / kBM;      // split tile among the tail
+  const int r = blockIdx.x - tt * kBM;  // row of the tile
+  const int tile = a.Qf + tt;
+  const int bh = tile / a.MT;
+  const int m = tile - bh * a.MT;
+  const int s0 = tt * a.pieces;
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+  float M = -INFINITY;
+  for (int p = 0; p < a.pieces; ++p) M = fmaxf(M, ml[(size_t)(s0 + p) * kBM + r].x);
+  float lsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int c = 4 * threadIdx.x;
+  for (int p = 0; p < a.pieces; ++p) {
+    const float2 e = ml[(size_t)(s0 + p) * kBM + r];
+    const float w = (e.x == -INFINITY) ? 0.f : exp2f(e.x - M);
+    lsum += w * e.y;
+    const float4 o = *reinterpret_cast<const float4*>(a.part_o + ((size_t)(s0 + p) * kBM + r) * D + c);
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const int pr = m * kBM + r;
+  const int f = pr / d.T_pad;
+  const int rr = pr - f * d.T_pad;
+  if (f >= d.Fc || rr >= d.T_f) return;
+  const int bb = bh / d.H;
+  const int h = bh - bb * d.H;
+  const size_t n_tok = (size_t)f * d.T_f + rr;
+  const float inv = (lsum > 0.f) ? 1.f / lsum : 0.f;
+  uint2 pk;
+  pk.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D + c) = pk;
+  if (threadIdx.x == 0 && a.lse) a.lse[(size_t)bh * d.Lq + n_tok] = (M + log2f(lsum)) * 0.69314718055994531f;
+}
+
 // ---- host side --------------------------------------------------------------
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -625,8 +713,12 @@ static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.MT, a.d.B * a.d.H);
+  const int tiles = a.MT * a.d.B * a.d.H;
+  dim3 grid(a.Qf + (tiles - a.Qf) * a.pieces);
   attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.Qf == tiles) return e;
+  attn_merge_kernel<D><<<(tiles - a.Qf) * kBM, D / 4, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -66,7 +66,15 @@ struct AttnArgs {
   int W, t0, t_lo, F;
   int MT;                    // 128-row query tiles per (b, h)
   float scale_log2;          // log2(e) / sqrt(D)
+  // Tail split: tiles 0 .. Qf-1 (b*h major, tile minor) run whole; each
+  // later tile is cut into `pieces` key ranges whose partial (O, max, sum)
+  // go to part_o / part_ml and are combined by a merge launch.
+  int Qf, pieces;
+  float* part_o;             // [piece slot][128][D] fp32, unnormalised
+  float* part_ml;            // [piece slot][128][2] running max (log2 units), sum
 };
+// Piece slots of the tail split (one per SM at most).
+constexpr int kAttnMaxPieces = 160;
 constexpr int kAttnMaxEntries = 4096;     // 64-row key units per CTA (two query tiles)
 constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
 

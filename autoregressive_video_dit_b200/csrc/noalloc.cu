@@ -16,7 +16,7 @@ namespace {
 // Fixed scratch: enough for the 1.3B-shaped 480P chunk (H = 12, D = 128,
 // 30 x 52 latent grid, 3 frames per chunk) with any budget up to 1024
 // candidate blocks; larger shapes are rejected.
-constexpr size_t kNoAllocScratchBytes = 24u << 20;  // 24 MiB
+constexpr size_t kNoAllocScratchBytes = 64u << 20;  // 64 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // The array's name is only a host-side stand-in; its device address is

@@ -221,8 +221,11 @@ int cva_hsa_select(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0
  * block_idx == NULL: every history frame's every block (dense).
  *   q_rot: bf16 [B][H][Fc*T_pad][D]; out: bf16 [B, Lq, H, D];
  *   lse: fp32 [B][H][Lq] or NULL.
- *   workspace: device scratch of cva_attn_workspace_bytes() bytes (may be
- *   NULL when that is 0).
+ *   workspace: device scratch of cva_attn_workspace_bytes() bytes (256-byte
+ *   aligned), or NULL. With it, the query tiles of the last, partial wave of
+ *   CTAs are cut into key-range pieces that fill the SMs and are merged by a
+ *   second launch (same result up to fp32 rounding order); without it every
+ *   tile runs whole. A smaller ws_bytes counts as NULL.
  * Tensor cores (tcgen05, accumulators in tensor memory), TMA tile loads
  * gathered by block index, fp32 online softmax. */
 int cva_attn_workspace_bytes(const cva_shape* shape, int32_t k_b_max, size_t* bytes);
@@ -249,7 +252,7 @@ int cva_chunk_attention(const void* q, const void* k, const void* v,
  * when they call, such as a plugin whose host runtime owns every allocation
  * and passes it only inputs and outputs, or a loop that forbids allocation
  * after start-up). Same arguments and results as cva_chunk_attention; the
- * scratch is one fixed 24 MiB array inside the library, held on every
+ * scratch is one fixed 64 MiB array inside the library, held on every
  * device that loads it until the process exits. Shapes and budgets that
  * need more return CVA_ENOMEM without launching. Calls never allocate or
  * free memory. The first call on a device looks up the array's address

@@ -233,14 +233,17 @@ def test_hsa_select_staged_c3_full_size(ops, chunk):
 
 # ---- step 5: attention ------------------------------------------------------------------
 
-def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0):
+def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0, split=False):
     import torch
     cache = _gpu_cache_from_oracle(ops, wl, run, t_begin)
+    ws = None
+    if split:  # with the scratch the tiles of the last partial wave run as key-range pieces
+        ws = torch.empty(ops.attn_workspace_bytes(cache.shape, 0), dtype=torch.uint8, device="cuda")
     qd = to_dev(f64_to_bits(_head_major(wl, run["q_rot"])))
     out = torch.full((wl.B, wl.Lq, wl.H, wl.D), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((wl.B, wl.H, wl.Lq), float("nan"), dtype=torch.float32, device="cuda")
     if blocks is None:
-        ops.blocksparse_attn_fwd(qd, cache, run["t0"], None, None, 0, out, lse)
+        ops.blocksparse_attn_fwd(qd, cache, run["t0"], None, None, 0, out, lse, ws)
     else:
         kb = blocks.shape[-1]
         # at least one element: an empty tensor has a NULL data pointer, which means "dense"
@@ -248,7 +251,7 @@ def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0):
         padded[..., :kb] = blocks
         bi = torch.from_numpy(padded).cuda()
         bc = torch.full(blocks.shape[:-1], kb, dtype=torch.int32, device="cuda")
-        ops.blocksparse_attn_fwd(qd, cache, run["t0"], bi, bc, kb, out, lse)
+        ops.blocksparse_attn_fwd(qd, cache, run["t0"], bi, bc, kb, out, lse, ws)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
     o_want, l_want = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, blocks, rows)
@@ -261,11 +264,12 @@ def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0):
     return mx, mean, rel
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("key", SMALL)
-def test_attention_staged(ops, key):
+def test_attention_staged(ops, key, split):
     wl = WORKLOADS[key]
     run = _oracle_run(wl, wl.chunk)
-    _check_attention(ops, wl, run, run["blocks"])
+    _check_attention(ops, wl, run, run["blocks"], split=split)
 
 
 @pytest.mark.parametrize("key", SMALL_SPARSE)
@@ -281,7 +285,7 @@ def test_attention_staged_c2_full_size_sampled(ops):
     heads = [3, 10]
     run = _oracle_run(wl, wl.chunk, heads)
     rows = sample_rows(wl, 2, np.random.default_rng(1))
-    _check_attention(ops, _sub(wl, heads), run, None, rows)
+    _check_attention(ops, _sub(wl, heads), run, None, rows, split=True)
 
 
 def test_attention_staged_c4_full_size_sampled(ops):

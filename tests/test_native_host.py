@@ -165,7 +165,9 @@ def test_workspace_bytes(ops):
     s = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
     r = lambda x: (x + 255) // 256 * 256
     bhq = wl.B * wl.H * wl.NQB
+    # attention scratch: partial O, max and sum of up to 160 key-range pieces
+    attn = r(160 * 128 * wl.D * 4) + r(160 * 128 * 2 * 4)
     want = (r(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r(bhq * wl.D * 4) + r(bhq * 8 * 4)
-            + r(bhq * 120 * 4) + r(bhq * 4))
+            + r(bhq * 120 * 4) + r(bhq * 4) + attn)
     assert ops.chunk_workspace_bytes(s, 8, 120) == want
-    assert ops.attn_workspace_bytes(s, 120) == 0
+    assert ops.attn_workspace_bytes(s, 120) == attn
