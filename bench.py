@@ -153,6 +153,19 @@ def block_lists(st):
     return raw.reshape(wl.B, wl.H, wl.NQB, st["k_b"]).astype(np.int64)
 
 
+def attention_launches(wl):
+    """Launches of the attention step: the kernel, plus the merge of the
+    tail-split pieces when the query tiles leave a partial last wave (the
+    library's rule: tail = tiles mod SMs, pieces = min(SMs // tail, 160 //
+    tail), split when pieces >= 2)."""
+    import torch
+    nsm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    tiles = -(-wl.Fc * wl.T_pad // 128) * wl.B * wl.H
+    tail = tiles % nsm
+    pieces = min(nsm // tail, 160 // tail) if tail else 0
+    return 2 if pieces >= 2 else 1
+
+
 def rope_bytes(wl):
     """Algorithmic HBM bytes of the rotate/append/pool stage: read Q, K, V and
     write rotated Q, rotated K and V (bf16)."""
@@ -510,7 +523,7 @@ def run_cuda(args):
                          "achieved": rb / (rope_avg * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": rb / (rope_avg * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
                          "algorithmic_bytes": rb},
-        "gpu_launches": n * (3 + (1 if (st["k_f"] >= 0 and st["F"] > 0) else 0)),
+        "gpu_launches": n * (2 + (1 if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
         "clocks": clocks,
     }
     if e2e:
