@@ -12,21 +12,22 @@
 // empty unit.
 //
 // Tensor memory holds two score buffers S0 and S1 (128 fp32 columns each,
-// P aliased onto the scores it came from) and the output accumulator O
-// (128 columns). With two score buffers the tensor core computes S(i+1)
-// while the softmax works on S(i), and PV(i) is followed right away by
-// S(i+2) into the buffer P(i) leaves: the MMAs of one tile overlap the
-// softmax of the next instead of waiting for it.
+// P aliased onto the scores it came from) and two output accumulators
+// O_even and O_odd (128 columns each). Key tile i's scores go to buffer
+// i mod 2 and its PV into O of the same parity. With two score buffers the
+// tensor core computes S(i+1) while the softmax works on S(i), and PV(i) is
+// followed right away by S(i+2) into the buffer P(i) leaves.
 //
 // Roles (384 threads):
-//   warps 0-7: softmax. Warps w and w + 4 own query rows 32 (w mod 4) ..
-//     + 31 (TMEM lanes; thread = row) and split the 128 key columns: warp
-//     w < 4 the first 64, warp w + 4 the last 64. They trade partial row
-//     maxima through shared memory (one named barrier per warp pair), then
-//     exp2 on the MUFU in fp32 with packed f32x2 arithmetic and write bf16 P
+//   warps 0-3 / 4-7: softmax of the even / odd key tiles. Warps w and w + 4
+//     own query rows 32 (w mod 4) .. + 31 (TMEM lanes; thread = row); each
+//     runs its own online softmax over its tiles (all 128 key columns) into
+//     its own O, so the two warps sharing a scheduler work on different tiles
+//     and never wait for each other. Masks, row maximum (3-input max), exp2
+//     on the MUFU in fp32 with packed f32x2 arithmetic, bf16 P written back
 //     over the S columns. O is rescaled in tensor memory only when the row
-//     maximum grows by more than 2^8, after PV(i-1) completed. Finally each
-//     warp normalises its half of O into bf16.
+//     maximum grows by more than 2^8 (S(i) completing implies PV(i-2) did).
+//     At the end the pair merges its two (O, max, sum) and writes bf16 O.
 //   warp 8 (one lane): TMA producer. Q once, then K and V of every tile in
 //     order into the ring slot t mod 2, each as soon as its slot is free,
 //     gathered by block index with one 64-row box per unit and 64-column
@@ -58,7 +59,7 @@ constexpr int kMmaWarp = 9;
 // 12 warps: registers are granted per group of four warps, so warps 10 and
 // 11 cost nothing extra; they only join the final barrier.
 constexpr int kAttnThreads = 384;
-constexpr uint32_t kTmemCols = 512;   // S0 at 0, S1 at 128, O at 256
+constexpr uint32_t kTmemCols = 512;   // S0 at 0, S1 at 128, O_even at 256, O_odd at 384
 constexpr uint32_t kOCol = 256;
 
 template <int D>
@@ -70,9 +71,9 @@ struct AttnSmem {
   static constexpr int kK = kQ + kTileBytes;                // slot s at + s * tile
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kEnt = kV + kStages * kTileBytes;
-  // softmax pair exchange: maxima [2 bufs][2 halves][128], sums [2][128], flags [3][2][4]
+  // softmax epilogue exchange: (max, sum) [2 parities][128 rows], flags [2][4]
   static constexpr int kRed = kEnt + kAttnMaxEntries * 4;
-  static constexpr int kBar = kRed + (2 * 2 * 128 + 2 * 128) * 4 + 3 * 2 * 4 * 4;
+  static constexpr int kBar = kRed + 2 * 128 * 8 + 2 * 4 * 4;
   static constexpr int kMisc = kBar + 32 * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
@@ -85,7 +86,7 @@ struct AttnSmem {
 // Barriers: S buffer b full / P written into it; K and V ring slots full and
 // free; PV done (every PV), O final; one for draining the tensor pipe.
 constexpr int kBarSFull = 0, kBarPFull = 2, kBarKFull = 4, kBarKEmpty = 6, kBarVFull = 8,
-              kBarVEmpty = 10, kBarQ = 12, kBarPVDone = 13, kBarODone = 14, kBarDrain = 15;
+              kBarVEmpty = 10, kBarQ = 12, kBarODone = 13, kBarDrain = 14;
 
 // Above this growth of the row maximum (log2 units) O is rescaled; below
 // it the stale maximum is kept, so P <= 2^8.
@@ -326,14 +327,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[kBarSFull + s], 1);
-      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps);
+      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps / 2);  // one warp set per buffer
       mbar_init(&bar[kBarKFull + s], 1);
       mbar_init(&bar[kBarKEmpty + s], 1);
       mbar_init(&bar[kBarVFull + s], 1);
       mbar_init(&bar[kBarVEmpty + s], 1);
     }
     mbar_init(&bar[kBarQ], 1);
-    mbar_init(&bar[kBarPVDone], 1);
     mbar_init(&bar[kBarODone], 1);
     mbar_init(&bar[kBarDrain], 1);
     *abort_flag = 0;
@@ -440,9 +440,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             !mbar_wait(&bar[kBarVFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err))
           break;
         tc_fence_after();
-        issue_pv<D>(tmem + kOCol, tmem + 128u * (i & 1), v_addr + (i & 1) * L::kTileBytes, i > 0);
+        // O_even / O_odd: the two softmax warp sets keep separate accumulators
+        issue_pv<D>(tmem + kOCol + 128u * (i & 1), tmem + 128u * (i & 1), v_addr + (i & 1) * L::kTileBytes,
+                    i >= 2);
         mma_commit(&bar[kBarVEmpty + (i & 1)]);
-        mma_commit(&bar[kBarPVDone]);
         if (i + 1 == N) mma_commit(&bar[kBarODone]);  // O final: the epilogue's wait
         if (i + 2 < N) ok = issue_score(i + 2);
       }
@@ -452,81 +453,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     const Dims& d = a.d;
-    const int quarter = warp & 3;        // TMEM lane quarter: rows 32 quarter ..
-    const int half = warp >> 2;          // key columns 64 half .. + 63
+    const int quarter = warp & 3;        // TMEM lane quarter: rows 32 quarter .. + 31
+    const int par = warp >> 2;           // this warp's key tiles: par, par + 2, par + 4, ...
     const int r = quarter * 32 + lane;   // query row of the tile = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t ocol = kOCol + 128u * par;  // this warp's O accumulator
     const int mbit = r >> 6;             // this row's bit in a unit mask (warp-uniform)
-    // red[buf][half][row]: partial row maxima; lsum[half][row]; okf[slot][half][quarter]
-    // (slots 0 and 1 per tile, slot 2 for the epilogue)
-    float* red = reinterpret_cast<float*>(smem + L::kRed);
-    float* lsum = red + 2 * 2 * 128;
-    volatile int* okf = reinterpret_cast<volatile int*>(lsum + 2 * 128);
+    // epilogue exchange: (max, sum) [2 parities][128 rows]; flags [2 parities][4 quarters]
+    float2* xch = reinterpret_cast<float2*>(smem + L::kRed);
+    volatile int* okf = reinterpret_cast<volatile int*>(xch + 2 * 128);
     const float sc = a.scale_log2;
     float m_used = -INFINITY;  // running maximum in scaled log2 units (possibly stale by < 8)
-    float l_run = 0.f;         // over this warp's half of the keys
+    float l_run = 0.f;
     bool ok = true;
-    for (int i = 0; i < N; ++i) {
-      const int buf = i & 1;
-      const uint32_t scol = 128u * buf + 64u * half;
-      bool mine = mbar_wait(&bar[kBarSFull + buf], (i >> 1) & 1, abort_flag, a.err);
-      mine = __all_sync(0xFFFFFFFFu, mine);
-      uint32_t s[2][32];
-      float pm = -INFINITY;
-      if (mine) {
-        tc_fence_after();
-        tmem_ld32(trow + scol, s[0]);
-        tmem_ld32(trow + scol + 32u, s[1]);
-        const uint32_t e = units[2 * i + half];
-        const int lim = ((e >> mbit) & 1u) ? (int)((e >> 8) & 0xFFu) : 0;
-        tmem_wait_ld();
-        if (lim < 64) {  // warp-uniform
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (32 * j + c >= lim) s[j][c] = __float_as_uint(-INFINITY);
-        }
-        float mx[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          mx[j] = fmaxf(__uint_as_float(s[j][0]), __uint_as_float(s[j][1]));
-#pragma unroll
-          for (int c = 2; c < 32; c += 2) mx[j] = max3f(mx[j], __uint_as_float(s[j][c]), __uint_as_float(s[j][c + 1]));
-        }
-        pm = fmaxf(mx[0], mx[1]);
-      }
-      // Both warps of the pair reach this barrier once per tile, whatever
-      // happened: it orders the maxima exchange, guarantees the partner has
-      // read its scores before P overwrites them, and lets both leave together.
-      red[(buf * 2 + half) * 128 + r] = pm;
-      if (lane == 0) okf[(buf * 2 + half) * 4 + quarter] = mine ? 1 : 0;
-      pair_sync(quarter);
-      ok = mine && okf[(buf * 2 + (half ^ 1)) * 4 + quarter] != 0;
+    for (int i = par; ok && i < N; i += 2) {
+      const int buf = i & 1;  // = par: S(i) and P(i) live in buffer par
+      ok = mbar_wait(&bar[kBarSFull + buf], (i >> 1) & 1, abort_flag, a.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
-      const float mt = fmaxf(pm, red[(buf * 2 + (half ^ 1)) * 128 + r]) * sc;  // -inf when nothing is valid
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(trow + 128u * buf + 32u * j, s[j]);
+      const uint32_t e0 = units[2 * i], e1 = units[2 * i + 1];
+      const int lim0 = ((e0 >> mbit) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
+      const int lim1 = ((e1 >> mbit) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
+      const bool full = (lim0 == 64) && (lim1 == 64);   // warp-uniform
+      tmem_wait_ld();
+      if (!full) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int lim = j < 2 ? lim0 - 32 * j : lim1 - 32 * (j - 2);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c >= lim) s[j][c] = __float_as_uint(-INFINITY);
+        }
+      }
+      // four independent chains of 3-input maxima, one per 32 columns
+      float mx[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        mx[j] = fmaxf(__uint_as_float(s[j][0]), __uint_as_float(s[j][1]));
+#pragma unroll
+        for (int c = 2; c < 32; c += 2) mx[j] = max3f(mx[j], __uint_as_float(s[j][c]), __uint_as_float(s[j][c + 1]));
+      }
+      const float mt = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;  // -inf when nothing is valid
       const bool need = mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt > -INFINITY);
-      if (__any_sync(0xFFFFFFFFu, need)) {  // same rows, same decision in both warps of the pair
+      if (__any_sync(0xFFFFFFFFu, need)) {
         const float m_new = need ? mt : m_used;
         const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
-        if (i > 0) {
-          // O must hold PV(0..i-1) before it is scaled. A failed wait skips
-          // the scaling but not the pair's barriers: the abort flag is up and
-          // both warps leave at the next tile's barrier.
-          bool done = mbar_wait(&bar[kBarPVDone], (i - 1) & 1, abort_flag, a.err);
-          done = __all_sync(0xFFFFFFFFu, done);
-          if (done) {
-            tc_fence_after();
+        if (i >= 2) {
+          // This warp's O holds PV(par .. i-2): S(i) was issued after PV(i-2)
+          // and reported complete, so that PV is done too.
 #pragma unroll 1
-            for (int j = 0; j < D / 32; ++j) {
-              const uint32_t oc = trow + kOCol + (uint32_t)(D / 2) * half + 16u * j;
-              uint32_t o[16];
-              tmem_ld16(oc, o);
-              tmem_wait_ld();
+          for (int j = 0; j < D / 16; ++j) {
+            uint32_t o[16];
+            tmem_ld16(trow + ocol + 16u * j, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              tmem_st16(oc, o);
-            }
+            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st16(trow + ocol + 16u * j, o);
           }
         }
         l_run *= alpha;
@@ -537,19 +523,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 nb2 = make_float2(-base, -base);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int h = 0; h < 4; ++h) {
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const float2 xv = ffma2(make_float2(__uint_as_float(s[j][2 * q]), __uint_as_float(s[j][2 * q + 1])),
+          const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
                                   sc2, nb2);
           const float2 p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
           if (q & 1) acc1 = fadd2(acc1, p);
           else acc0 = fadd2(acc0, p);
           pk[q] = cvt_bf16x2(p.x, p.y);
         }
-        // bf16 pairs: keys 64 half + 32 j .. go to packed columns 32 half + 16 j
-        tmem_st16(trow + 128u * buf + 32u * half + 16u * j, pk);
+        tmem_st16(trow + 128u * buf + 16u * h, pk);
       }
       l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
@@ -557,69 +542,83 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&bar[kBarPFull + buf]);
     }
     // ------------------------------------------------------------ epilogue
-    bool fin = false;
-    if (ok) {
-      fin = N == 0 || mbar_wait(&bar[kBarODone], 0, abort_flag, a.err);  // an empty piece has no PV
-      fin = __all_sync(0xFFFFFFFFu, fin);
-      lsum[half * 128 + r] = l_run;
-      if (lane == 0) okf[(2 * 2 + half) * 4 + quarter] = fin ? 1 : 0;
-      pair_sync(quarter);  // both warps of the pair got here: both left the loop with ok
-      fin = fin && okf[(2 * 2 + (half ^ 1)) * 4 + quarter] != 0;
-    }
-    if (fin && slot >= 0) {
-      // A piece of a split tile: raw O (relative to the running maximum),
-      // the maximum and the sum, for the merge launch.
+    // Both warps of a row range always get here and meet once: the two
+    // partial softmaxes (even and odd key tiles) are merged.
+    bool fin = ok && (N == 0 || mbar_wait(&bar[kBarODone], 0, abort_flag, a.err));  // empty piece: no PV
+    fin = __all_sync(0xFFFFFFFFu, fin);
+    xch[par * 128 + r] = make_float2(m_used, l_run);
+    if (lane == 0) okf[par * 4 + quarter] = fin ? 1 : 0;
+    pair_sync(quarter);
+    fin = fin && okf[(par ^ 1) * 4 + quarter] != 0;
+    if (fin) {
       if (N > 0) tc_fence_after();
-      const float l_tot = l_run + lsum[(half ^ 1) * 128 + r];
-      float* po = a.part_o + ((size_t)slot * kBM + r) * D + (D / 2) * half;
-#pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
-        uint32_t o[32];
-        if (N > 0) {
-          tmem_ld32(trow + kOCol + (uint32_t)(D / 2) * half + 32u * i, o);
-          tmem_wait_ld();
-        } else {
+      const float2 e0 = xch[r], e1 = xch[128 + r];  // parities 0 and 1
+      const float M = fmaxf(e0.x, e1.x);
+      const float w0 = (e0.x == -INFINITY) ? 0.f : fast_exp2(e0.x - M);
+      const float w1 = (e1.x == -INFINITY) ? 0.f : fast_exp2(e1.x - M);
+      const float l_tot = e0.y * w0 + e1.y * w1;
+      // this warp writes columns [D/2 par, D/2 par + D/2) from both accumulators
+      const uint32_t c0 = (uint32_t)(D / 2) * par;
+      auto merged = [&](int i, uint32_t (&o)[32]) {  // columns c0 + 32 i .. + 31, relative to M
+        if (N == 0) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
+          return;
         }
-        float4* dst = reinterpret_cast<float4*>(po + 32 * i);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                               __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-      }
-      if (half == 0)
-        reinterpret_cast<float2*>(a.part_ml)[(size_t)slot * kBM + r] = make_float2(m_used, l_tot);
-    } else if (fin) {
-      tc_fence_after();
-      const float l_tot = l_run + lsum[(half ^ 1) * 128 + r];
-      const int pr = m * kBM + r;  // row in the padded chunk
-      const int f = pr / d.T_pad;
-      const int rr = pr - f * d.T_pad;
-      const bool row_ok = (f < d.Fc) && (rr < d.T_f);
-      const int bb = bh / d.H;
-      const int h = bh - bb * d.H;
-      const size_t n_tok = (size_t)f * d.T_f + rr;
-      const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-      uint16_t* orow = a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D + (D / 2) * half;
-#pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
-        uint32_t o[32];
-        tmem_ld32(trow + kOCol + (uint32_t)(D / 2) * half + 32u * i, o);
+        uint32_t o1[32];
+        tmem_ld32(trow + kOCol + c0 + 32u * i, o);
+        tmem_ld32(trow + kOCol + 128u + c0 + 32u * i, o1);
         tmem_wait_ld();
-        if (row_ok) {
-          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            pk[c] = cvt_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * i);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int c = 0; c < 32; ++c) {
+          // an accumulator no PV wrote (w = 0) holds garbage: never multiply it
+          const float a0 = w0 > 0.f ? __uint_as_float(o[c]) * w0 : 0.f;
+          const float a1 = w1 > 0.f ? __uint_as_float(o1[c]) * w1 : 0.f;
+          o[c] = __float_as_uint(a0 + a1);
         }
+      };
+      if (slot >= 0) {
+        // A piece of a split tile: O relative to M, M and the sum, for the merge launch.
+        float* po = a.part_o + ((size_t)slot * kBM + r) * D + c0;
+#pragma unroll
+        for (int i = 0; i < D / 64; ++i) {
+          uint32_t o[32];
+          merged(i, o);
+          float4* dst = reinterpret_cast<float4*>(po + 32 * i);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+        if (par == 0) reinterpret_cast<float2*>(a.part_ml)[(size_t)slot * kBM + r] = make_float2(M, l_tot);
+      } else {
+        const int pr = m * kBM + r;  // row in the padded chunk
+        const int f = pr / d.T_pad;
+        const int rr = pr - f * d.T_pad;
+        const bool row_ok = (f < d.Fc) && (rr < d.T_f);
+        const int bb = bh / d.H;
+        const int h = bh - bb * d.H;
+        const size_t n_tok = (size_t)f * d.T_f + rr;
+        const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+        uint16_t* orow = a.out + (((size_t)bb * d.Lq + n_tok) * d.H + h) * D + c0;
+#pragma unroll
+        for (int i = 0; i < D / 64; ++i) {
+          uint32_t o[32];
+          merged(i, o);
+          if (row_ok) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              pk[c] = cvt_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * i);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (row_ok && par == 0 && a.lse)
+          a.lse[(size_t)bh * d.Lq + n_tok] = (M + log2f(l_tot)) * 0.69314718055994531f;
       }
-      if (row_ok && half == 0 && a.lse)
-        a.lse[(size_t)bh * d.Lq + n_tok] = (m_used + log2f(l_tot)) * 0.69314718055994531f;
     }
   }
 
