@@ -28,6 +28,7 @@ Modules:
 * :mod:`oracle.hsa`       -- pooling, two-level top-k selection, budgets.
 * :mod:`oracle.attention` -- chunk attention over an explicit key set.
 * :mod:`oracle.path`      -- a frame cache and the whole per-chunk path.
+* :mod:`oracle.qkv`       -- QKV projection followed by Causal-RoPE.
 
 Where the pages leave a step open the oracle takes one reading, named in
 each function's docstring. Functions whose behaviour rests on such a

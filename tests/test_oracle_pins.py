@@ -368,3 +368,58 @@ def test_cag_other_workloads():
     assert _b(WORKLOADS["c5"], 2, 3) == (3, 15)
     assert _b(WORKLOADS["c2"], 7, 18) == (18, 450)         # dense
     assert _b(WORKLOADS["c1s"], 4, 9) == (4, 4)
+
+
+# ---- QKV projection + Causal-RoPE (section 2C operator fusion) ----------------
+
+def test_qkv_identity_weight_selects_q_k_v_slices():
+    # C = 3HD and W = I: q, k, v are consecutive H*D slices of x, head-major
+    # inside each; q and k then rotate exactly like the pinned rope_chunk.
+    from oracle import qkv
+    rng = np.random.default_rng(5)
+    H, D, Fh, Fw, Fc, t0 = 2, 6, 2, 3, 2, 4
+    Lq = Fc * Fh * Fw
+    x = rng.standard_normal((1, Lq, 3 * H * D))
+    q, k, v = qkv.project(x, np.eye(3 * H * D), H, D)
+    np.testing.assert_array_equal(q, x[:, :, :H * D].reshape(1, Lq, H, D))
+    np.testing.assert_array_equal(k, x[:, :, H * D:2 * H * D].reshape(1, Lq, H, D))
+    np.testing.assert_array_equal(v, x[:, :, 2 * H * D:].reshape(1, Lq, H, D))
+    qr, kr, vv = qkv.qkv_rope(x, np.eye(3 * H * D), H, D, Fh, Fw, Fc, t0)
+    np.testing.assert_allclose(qr, rope.rope_chunk(q, Fh, Fw, Fc, t0), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(kr, rope.rope_chunk(k, Fh, Fw, Fc, t0), rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(vv, v)
+
+
+def test_qkv_projection_brute_force():
+    # y[b, n, o] = sum_c x[b, n, c] * W[o, c], written out with loops
+    from oracle import qkv
+    rng = np.random.default_rng(6)
+    B, Lq, C, H, D = 2, 3, 5, 1, 2
+    x = rng.standard_normal((B, Lq, C))
+    w = rng.standard_normal((3 * H * D, C))
+    q, k, v = qkv.project(x, w, H, D)
+    y = np.stack([q, k, v], axis=2).reshape(B, Lq, 3 * H * D)
+    for b in range(B):
+        for n in range(Lq):
+            for o in range(3 * H * D):
+                s = 0.0
+                for c in range(C):
+                    s += x[b, n, c] * w[o, c]
+                assert abs(y[b, n, o] - s) < 1e-12
+
+
+def test_qkv_rotation_after_projection_keeps_pair_norms_of_the_projection():
+    # rotation is applied to the projected q (not to x): pair norms of q_rot
+    # equal those of x W_q^T, and v is untouched by any rotation
+    from oracle import qkv
+    rng = np.random.default_rng(7)
+    H, D, Fh, Fw, Fc, t0 = 2, 8, 2, 2, 3, 9
+    x = rng.standard_normal((1, Fc * Fh * Fw, 16))
+    w = rng.standard_normal((3 * H * D, 16))
+    q, k, v = qkv.project(x, w, H, D)
+    qr, kr, vv = qkv.qkv_rope(x, w, H, D, Fh, Fw, Fc, t0)
+    n = lambda a: a[..., 0::2] ** 2 + a[..., 1::2] ** 2
+    np.testing.assert_allclose(n(qr), n(q), rtol=1e-12)
+    np.testing.assert_allclose(n(kr), n(k), rtol=1e-12)
+    np.testing.assert_array_equal(vv, v)
+    assert not np.allclose(qr, q)
