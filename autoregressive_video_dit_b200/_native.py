@@ -71,6 +71,8 @@ _SIGS = {
     "cva_rope3d_apply": (c_int32, [c_void_p, c_void_p, P(RopeTables), P(Shape), c_int32, c_int32, c_void_p]),
     "cva_kv_append": (c_int32, [c_void_p, c_void_p, P(KVCache), P(RopeTables), c_int32, c_void_p]),
     "cva_history_frames": (c_int32, [P(KVCache), c_int32, P(c_int32), P(c_int32)]),
+    "cva_qkv_rope_append": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
+                                      c_void_p, c_void_p, c_void_p]),
     "cva_hsa_compress": (c_int32, [c_void_p, P(Shape), c_void_p, c_void_p, c_void_p]),
     "cva_hsa_select": (c_int32, [c_void_p, P(KVCache), c_int32, c_int32, c_int32, c_void_p,
                                  c_void_p, c_void_p, c_void_p]),
@@ -281,6 +283,14 @@ def kv_append(k, v, cache: DeviceKVCache, tables: Optional[DeviceRopeTables], t0
     check(lib.cva_kv_append(_ptr(k), _ptr(v), ctypes.byref(cache.struct),
                             None if tables is None else ctypes.byref(tables.struct), t0,
                             _stream(stream)))
+
+
+def qkv_rope_append(x, w_qkv, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, q_rot,
+                    qpool_blk=None, stream=None) -> None:
+    """x: bf16 [B, Lq, C]; w_qkv: bf16 [3*H*D, C]; q_rot: bf16 [B][H][Fc*T_pad][D] (output)."""
+    check(lib.cva_qkv_rope_append(_ptr(x), _ptr(w_qkv), int(x.shape[-1]), ctypes.byref(cache.struct),
+                                  ctypes.byref(tables.struct), t0, _ptr(q_rot), _ptr(qpool_blk),
+                                  _stream(stream)))
 
 
 def hsa_compress(q_rot, shape: Shape, qpool_blk, qpool_frm=None, stream=None) -> None:

@@ -385,6 +385,44 @@ int cva_kv_append(const void* k, const void* v, const cva_kv_cache* cache,
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "kv_append frame pool launch");
 }
 
+int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden, const cva_kv_cache* cache,
+                        const cva_rope_tables* tables, int32_t t0, void* q_rot, float* qpool_blk,
+                        cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!x || !w_qkv || !q_rot || !tables) return fail(CVA_EINVAL, "x, w_qkv, q_rot or tables is NULL");
+  if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(q_rot, 16))
+    return fail(CVA_EINVAL, "x, w_qkv and q_rot must be 16-byte aligned");
+  if (hidden < 64 || hidden % 64) return fail(CVA_ENOTSUP, "hidden %d must be a positive multiple of 64", hidden);
+  const Dims d = make_dims(cache->shape);
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  rc = check_tables(tables, d, t0);
+  if (rc) return rc;
+  QkvArgs a = {};
+  a.d = d;
+  a.C = hidden;
+  a.t0 = t0;
+  a.W = cache->window;
+  a.tab = make_tab(tables, d.D);
+  a.q_rot = static_cast<uint16_t*>(q_rot);
+  a.k_cache = static_cast<uint16_t*>(cache->k);
+  a.v_cache = static_cast<uint16_t*>(cache->v);
+  a.qpool = qpool_blk;
+  a.kpool_blk = cache->kpool_blk;
+  a.MT = (d.Fc * d.T_pad + 127) / 128;
+  a.NT = (3 * d.H * d.D + 255) / 256;
+  a.err = device_error_word();
+  if (a.MT > 65535) return fail(CVA_ENOTSUP, "padded chunk rows %d too many", d.Fc * d.T_pad);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const char* why = "";
+  cudaError_t e = launch_qkv_rope(a, x, w_qkv, s, &why);
+  if (e == cudaErrorInvalidValue && why[0]) return fail(CVA_ELAUNCH, "qkv_rope_append: %s", why);
+  if (e != cudaSuccess) return cuda_fail(e, "qkv_rope_append launch");
+  FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
+  e = launch_frame_pool(fp, s);
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "qkv_rope_append frame pool launch");
+}
+
 int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk, float* qpool_frm,
                      cva_stream_t stream) {
   int rc = check_shape(shape);

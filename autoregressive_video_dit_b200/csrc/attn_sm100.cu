@@ -689,8 +689,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 3D bf16 map over [d2][d1][d0] (d0 innermost), box (64 columns, box1 rows), 128 B swizzle.
-static bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                     uint32_t box1) {
+bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint32_t box1) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {d0, d1, d2};

@@ -82,6 +82,28 @@ constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
 cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
                              const void* cache_v, cudaStream_t stream, const char** why);
 
+// Tiled TMA descriptor of a bf16 tensor [d2][d1][d0] (d0 innermost) with a
+// box of 64 x box1 elements and 128-byte swizzle (attn_sm100.cu).
+bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
+
+// ---- QKV projection + Causal-RoPE + append + block pooling (qkv_rope.cu) --
+struct QkvArgs {
+  Dims d;
+  int C;                     // hidden size (multiple of 64)
+  int t0, W;                 // chunk start frame, cache window
+  RopeTab tab;
+  uint16_t* q_rot;           // [B][H][Fc*T_pad][D]
+  uint16_t* k_cache;         // [B][H][W][T_pad][D]
+  uint16_t* v_cache;
+  float* qpool;              // [B][H][NQB][D] block means of q_rot, or nullptr
+  float* kpool_blk;          // [B][H][W][nb][D] block means of k_rot
+  int MT;                    // 128-row tiles over the padded rows of the chunk
+  int NT;                    // 256-column tiles over the 3*H*D projection outputs
+  int* err;
+};
+cudaError_t launch_qkv_rope(const QkvArgs& a, const void* x, const void* w, cudaStream_t stream,
+                            const char** why);
+
 // Sets the thread-local message cva_last_error() returns; returns `code`.
 int report_error(int code, const char* msg);
 

@@ -220,3 +220,16 @@ def chunk_inputs(wl: Workload, chunk: Optional[int] = None, layer: int = 0,
         "q": bf16_bits(q32), "k": bf16_bits(k32), "v": bf16_bits(v32),
         "chunk": c, "layer": layer, "t0": wl.t0_of(c),
     }
+
+
+def hidden_inputs(wl: Workload, hidden: int, chunk: Optional[int] = None, layer: int = 0) -> dict:
+    """Hidden states of one chunk and a projection weight for the fused QKV
+    step: ``x [B, Lq, C]`` N(0, 1) and ``w [3 H D, C]`` N(0, 1/C) (so the
+    projected q, k, v are about N(0, 1)), drawn in fp32 from the chunk's
+    seed (offset so they differ from :func:`chunk_inputs`) and rounded once
+    to bfloat16. Returns the bits (uint16) under ``x`` and ``w``."""
+    c = wl.chunk if chunk is None else chunk
+    rng = np.random.Generator(np.random.PCG64(seed_for(wl.config_index, c, layer) + 500))
+    x32 = rng.standard_normal((wl.B, wl.Lq, hidden), dtype=np.float32)
+    w32 = rng.standard_normal((3 * wl.H * wl.D, hidden), dtype=np.float32) / np.float32(np.sqrt(hidden))
+    return {"x": bf16_bits(x32), "w": bf16_bits(w32)}

@@ -234,6 +234,28 @@ int cva_blocksparse_attn_fwd(const void* q_rot, const cva_kv_cache* cache, int32
                              int32_t k_b_max, void* out, float* lse, void* workspace,
                              size_t ws_bytes, cva_stream_t stream);
 
+/* ---- QKV projection fused with steps 1-3 ----------------------------------
+ * "Accelerating Video Generation Inference with Sequential-Parallel 3D
+ * Positional Encoding Using a Global Time Index", section 2C (operator
+ * fusion: the QKV projection and Causal-RoPE in one kernel) with the global
+ * time index of section 2B.
+ *
+ * y = x W^T for the chunk's tokens, on the tensor cores (fp32 accumulate):
+ *   x:     bf16 [B, Lq, C], C = hidden (a multiple of 64, >= 64);
+ *   w_qkv: bf16 [3*H*D, C], rows: q heads 0..H-1 (D rows each), then the k
+ *          heads, then the v heads; no bias.
+ * q and k are rotated like cva_rope3d_apply (temporal coordinate t0 + f),
+ * in fp32 from the accumulator, and rounded once to bf16. Writes
+ *   q_rot:     bf16 [B][H][Fc*T_pad][D], pad rows zero (the attention's Q);
+ *   qpool_blk: fp32 [B][H][NQB][D] block means of the stored q, or NULL;
+ * and appends k and v to the cache slots of frames t0 .. t0+Fc-1 exactly as
+ * cva_kv_append does (pad rows zero, block and frame means of the stored
+ * k). x, w_qkv and q_rot must be 16-byte aligned. Two launches: the fused
+ * projection kernel and the frame pooling of the new cache frames. */
+int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden,
+                        const cva_kv_cache* cache, const cva_rope_tables* tables,
+                        int32_t t0, void* q_rot, float* qpool_blk, cva_stream_t stream);
+
 /* ---- fused chunk call ---------------------------------------------------- */
 
 /* Steps 1-5 for one chunk: RoPE(Q) with Q pooling, RoPE(K)+append+K pooling,
