@@ -25,8 +25,14 @@
 // shuffles, then the warps of the block in order), as the attention's
 // selection step needs them.
 //
+// Persistent: one CTA per SM walks its tiles (grouped order for L2 reuse);
+// the accumulator is double-buffered in tensor memory (2 x 256 columns), so
+// the MMAs of the next tile run while the epilogue rotates and stores the
+// previous one. The epilogue warps also stage the cos/sin rows of the chunk
+// in shared memory before the first tile.
+//
 // Roles (192 threads): warps 0-3 epilogue, warp 4 TMA producer (one lane),
-// warp 5 MMA issuer (one lane; also allocates the 256 TMEM columns). Every
+// warp 5 MMA issuer (one lane; also allocates the 512 TMEM columns). Every
 // wait is bounded (4 s, then CVA_DEV_TIMEOUT and every role leaves).
 #include <cudaTypedefs.h>
 
@@ -41,6 +47,7 @@ constexpr int kQkvStages = 4;
 constexpr int kQkvThreads = 192;
 constexpr int kQkvProducerWarp = 4;
 constexpr int kQkvMmaWarp = 5;
+constexpr int kQkvGroupM = 8;
 
 struct QkvSmem {
   static constexpr int kABytes = kQkvBM * kQkvBK * 2;  // 16 KB: two 64-row boxes
@@ -49,14 +56,19 @@ struct QkvSmem {
   static constexpr int kA = 0;                         // stage s at + s * kStageBytes
   static constexpr int kB = kABytes;
   static constexpr int kRed = kQkvStages * kStageBytes;  // [2][4 warps][32] column sums
-  static constexpr int kBar = kRed + 2 * 4 * 32 * 4;
+  static constexpr int kTab = kRed + 2 * 4 * 32 * 4;       // cos/sin tables of the chunk
+  static constexpr int kTabFloats = 7168;
+  static constexpr int kBar = kTab + kTabFloats * 4;
   static constexpr int kMisc = kBar + 16 * 8;
   static constexpr int kBytes = kMisc + 32;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory of one CTA");
 };
 
-// Barriers: stage s full / empty, accumulator done.
-constexpr int kQBarFull = 0, kQBarEmpty = kQkvStages, kQBarAcc = 2 * kQkvStages;
+// Barriers: stage s full / empty; accumulator buffer u full (MMAs done) /
+// empty (epilogue done reading it).
+constexpr int kQBarFull = 0, kQBarEmpty = kQkvStages, kQBarAccFull = 2 * kQkvStages,
+              kQBarAccEmpty = 2 * kQkvStages + 2;
 
 __device__ __forceinline__ void qkv_epi_sync() {  // the 4 epilogue warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -70,9 +82,20 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const Dims& d = a.d;
-  const int nt = blockIdx.x;   // 256-column tile of y
-  const int mt = blockIdx.y;   // 128 padded rows
-  const int b = blockIdx.z;
+  // Persistent: CTA c takes tiles c, c + gridDim.x, ... Tile order: per
+  // batch, groups of kQkvGroupM row tiles; inside a group the column tile is
+  // the slower index, so the CTAs that run together share a few weight
+  // tiles and a few row tiles (both stay in L2).
+  const int ntiles = d.B * a.MT * a.NT;
+  auto decode = [&](int id, int& b, int& mt, int& nt) {
+    b = id / (a.MT * a.NT);
+    id -= b * (a.MT * a.NT);
+    const int g = id / (kQkvGroupM * a.NT);
+    const int r0 = id - g * (kQkvGroupM * a.NT);
+    const int gm = min(kQkvGroupM, a.MT - g * kQkvGroupM);
+    nt = r0 / gm;
+    mt = g * kQkvGroupM + (r0 - nt * gm);
+  };
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -86,12 +109,15 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       mbar_init(&bar[kQBarFull + s], 1);
       mbar_init(&bar[kQBarEmpty + s], 1);
     }
-    mbar_init(&bar[kQBarAcc], 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bar[kQBarAccFull + u], 1);
+      mbar_init(&bar[kQBarAccEmpty + u], 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == kQkvMmaWarp) {
-    tmem_alloc(tmem_slot, kQkvBN);
+    tmem_alloc(tmem_slot, 2 * kQkvBN);  // two accumulator buffers
     tmem_relinquish();
   }
   tc_fence_before();
@@ -104,25 +130,32 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmW);
-      // token row of each 64-row half of the tile (Lq: past the end, zero-filled)
-      int tok[2];
-      for (int h = 0; h < 2; ++h) {
-        const int pr = mt * kQkvBM + 64 * h;
-        const int f = pr / d.T_pad;
-        tok[h] = (f < d.Fc) ? f * d.T_f + (pr - f * d.T_pad) : d.Lq;
-      }
-      int issued = 0;
-      for (int k = 0; k < KT; ++k) {
-        const int s = k % kQkvStages;
-        if (k >= kQkvStages &&
-            !mbar_wait(&bar[kQBarEmpty + s], ((k / kQkvStages) - 1) & 1, abort_flag, a.err))
-          break;
-        ++issued;
-        uint8_t* st = smem + s * L::kStageBytes;
-        mbar_arrive_expect_tx(&bar[kQBarFull + s], L::kStageBytes);
-        tma_load_3d(st + L::kA, &tmX, &bar[kQBarFull + s], k * kQkvBK, tok[0], b);
-        tma_load_3d(st + L::kA + 8192, &tmX, &bar[kQBarFull + s], k * kQkvBK, tok[1], b);
-        tma_load_3d(st + L::kB, &tmW, &bar[kQBarFull + s], k * kQkvBK, nt * kQkvBN, 0);
+      int issued = 0;  // k-steps over all of this CTA's tiles: stage issued % S
+      bool ok = true;
+      for (int id = blockIdx.x; ok && id < ntiles; id += gridDim.x) {
+        int b, mt, nt;
+        decode(id, b, mt, nt);
+        // token row of each 64-row half of the tile (Lq: past the end, zero-filled)
+        int tok[2];
+        for (int h = 0; h < 2; ++h) {
+          const int pr = mt * kQkvBM + 64 * h;
+          const int f = pr / d.T_pad;
+          tok[h] = (f < d.Fc) ? f * d.T_f + (pr - f * d.T_pad) : d.Lq;
+        }
+        for (int k = 0; k < KT; ++k) {
+          const int s = issued % kQkvStages;
+          if (issued >= kQkvStages &&
+              !mbar_wait(&bar[kQBarEmpty + s], ((issued / kQkvStages) - 1) & 1, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          ++issued;
+          uint8_t* st = smem + s * L::kStageBytes;
+          mbar_arrive_expect_tx(&bar[kQBarFull + s], L::kStageBytes);
+          tma_load_3d(st + L::kA, &tmX, &bar[kQBarFull + s], k * kQkvBK, tok[0], b);
+          tma_load_3d(st + L::kA + 8192, &tmX, &bar[kQBarFull + s], k * kQkvBK, tok[1], b);
+          tma_load_3d(st + L::kB, &tmW, &bar[kQBarFull + s], k * kQkvBK, nt * kQkvBN, 0);
+        }
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
         for (int k = (issued > kQkvStages ? issued - kQkvStages : 0); k < issued; ++k) {
@@ -137,35 +170,63 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kId = idesc_bf16_f32(kQkvBM, kQkvBN, 0, 0);  // both K-major
       bool ok = true;
-      for (int k = 0; ok && k < KT; ++k) {
-        const int s = k % kQkvStages;
-        ok = mbar_wait(&bar[kQBarFull + s], (k / kQkvStages) & 1, abort_flag, a.err);
-        if (!ok) break;
+      int used = 0;  // k-steps consumed over all tiles
+      for (int id = blockIdx.x, lt = 0; ok && id < ntiles; id += gridDim.x, ++lt) {
+        const int u = lt & 1;  // accumulator buffer of this tile
+        // the epilogue must have read the tile that used buffer u before
+        if (lt >= 2 && !mbar_wait(&bar[kQBarAccEmpty + u], ((lt >> 1) - 1) & 1, abort_flag, a.err)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * L::kStageBytes + L::kA);
-        const uint32_t b_addr = smem_u32(smem + s * L::kStageBytes + L::kB);
+        const uint32_t acc = tmem + (uint32_t)(u * kQkvBN);
+        for (int k = 0; k < KT; ++k, ++used) {
+          const int s = used % kQkvStages;
+          ok = mbar_wait(&bar[kQBarFull + s], (used / kQkvStages) & 1, abort_flag, a.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::kStageBytes + L::kA);
+          const uint32_t b_addr = smem_u32(smem + s * L::kStageBytes + L::kB);
 #pragma unroll
-        for (int kk = 0; kk < kQkvBK / 16; ++kk)
-          mma_ss(tmem, smem_desc_sw128(a_addr + 32u * kk, 16, 1024), smem_desc_sw128(b_addr + 32u * kk, 16, 1024),
-                 kId, (k > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar[kQBarEmpty + s]);
+          for (int kk = 0; kk < kQkvBK / 16; ++kk)
+            mma_ss(acc, smem_desc_sw128(a_addr + 32u * kk, 16, 1024), smem_desc_sw128(b_addr + 32u * kk, 16, 1024),
+                   kId, (k > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar[kQBarEmpty + s]);
+        }
+        if (ok) mma_commit(&bar[kQBarAccFull + u]);
       }
-      // also after an abort, so the epilogue does not wait out its limit; the
-      // latched error marks the result invalid
-      mma_commit(&bar[kQBarAcc]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int r = tid;  // row of the tile = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     volatile int* okw = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [4]
-    bool ok = mbar_wait(&bar[kQBarAcc], 0, abort_flag, a.err);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    if (lane == 0) okw[warp] = ok ? 1 : 0;
-    qkv_epi_sync();  // the four warps take the same path through the barriers below
-    ok = okw[0] && okw[1] && okw[2] && okw[3];
-    if (ok) {
+    // While the MMAs run: copy the cos/sin rows the chunk needs into shared
+    // memory: [cos_t, sin_t] of frames t0 .. t0+Fc-1, then [cos_h, sin_h]
+    // (Fh rows), then [cos_w, sin_w] (Fw rows).
+    const int nt_f = d.Fc * a.tab.pt, nh_f = d.Fh * a.tab.ph, nw_f = d.Fw * a.tab.pw;
+    const bool stab = 2 * (nt_f + nh_f + nw_f) <= L::kTabFloats;  // uniform
+    float* tb = reinterpret_cast<float*>(smem + L::kTab);
+    if (stab) {
+      const float* src_t = a.tab.cos_t + (size_t)a.t0 * a.tab.pt;
+      const float* src_ts = a.tab.sin_t + (size_t)a.t0 * a.tab.pt;
+      for (int i = tid; i < nt_f; i += 128) { tb[i] = src_t[i]; tb[nt_f + i] = src_ts[i]; }
+      float* th = tb + 2 * nt_f;
+      for (int i = tid; i < nh_f; i += 128) { th[i] = a.tab.cos_h[i]; th[nh_f + i] = a.tab.sin_h[i]; }
+      float* tw = th + 2 * nh_f;
+      for (int i = tid; i < nw_f; i += 128) { tw[i] = a.tab.cos_w[i]; tw[nw_f + i] = a.tab.sin_w[i]; }
+    }
+    qkv_epi_sync();
+    for (int id = blockIdx.x, lt = 0; id < ntiles; id += gridDim.x, ++lt) {
+      int b, mt, nt;
+      decode(id, b, mt, nt);
+      const int u = lt & 1;  // accumulator buffer of this tile
+      bool ok = mbar_wait(&bar[kQBarAccFull + u], (lt >> 1) & 1, abort_flag, a.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (lane == 0) okw[warp] = ok ? 1 : 0;
+      qkv_epi_sync();  // the four warps take the same path through the barriers below
+      ok = okw[0] && okw[1] && okw[2] && okw[3];
+      qkv_epi_sync();  // okw is rewritten for the next tile
+      if (!ok) break;
       tc_fence_after();
+      const uint32_t tacc = trow + (uint32_t)(u * kQkvBN);
       const int pr = mt * kQkvBM + r;  // padded row in the chunk
       const int f = pr / d.T_pad;
       const int rr = pr - f * d.T_pad;
@@ -175,6 +236,17 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       const int slot = t % a.W;
       const int hh = rr / d.Fw;
       const int ww = rr - hh * d.Fw;
+      // table row offsets of this row (position 0 for rows that are not
+      // tokens); the staged time table starts at frame t0
+      const size_t t_off = valid ? (size_t)(stab ? f : t) * a.tab.pt : 0;
+      const size_t h_off = valid ? (size_t)hh * a.tab.ph : 0;
+      const size_t w_off = valid ? (size_t)ww * a.tab.pw : 0;
+      const float* tct = stab ? tb : a.tab.cos_t;
+      const float* tst = stab ? tb + nt_f : a.tab.sin_t;
+      const float* tch = stab ? tb + 2 * nt_f : a.tab.cos_h;
+      const float* tsh = stab ? tb + 2 * nt_f + nh_f : a.tab.sin_h;
+      const float* tcw = stab ? tb + 2 * nt_f + 2 * nh_f : a.tab.cos_w;
+      const float* tsw = stab ? tb + 2 * nt_f + 2 * nh_f + nw_f : a.tab.sin_w;
       const int j = rr / d.blk;                  // block of the frame
       const int jb = f * d.nb + j;               // query block of the chunk
       const float vcnt = (float)((j == d.nb - 1) ? d.tail : d.blk);
@@ -190,33 +262,38 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
         const int head = rem / d.D;
         const int d0 = rem - head * d.D;
         uint32_t o[32];
-        tmem_ld32(trow + 32u * cc, o);
+        tmem_ld32(tacc + 32u * cc, o);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (which < 2) {
+          // cos/sin of the chunk's 16 pairs: all loads issued before any use
+          // (pad rows use position 0; their output is zero anyway)
+          float cs[16], sn[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float y0 = __uint_as_float(o[2 * i]), y1 = __uint_as_float(o[2 * i + 1]);
-          if (which < 2) {
-            const int p = (d0 >> 1) + i;
+          for (int i = 0; i < 16; ++i) {
+            const int p = (d0 >> 1) + i;       // warp-uniform
             const float* ct;
             const float* stb;
-            int pos, idx, stride;
+            size_t off;
             if (p < a.tab.pt) {
-              ct = a.tab.cos_t; stb = a.tab.sin_t; pos = t; idx = p; stride = a.tab.pt;
+              ct = tct; stb = tst; off = t_off + p;
             } else if (p < a.tab.pt + a.tab.ph) {
-              ct = a.tab.cos_h; stb = a.tab.sin_h; pos = hh; idx = p - a.tab.pt; stride = a.tab.ph;
+              ct = tch; stb = tsh; off = h_off + (p - a.tab.pt);
             } else {
-              ct = a.tab.cos_w; stb = a.tab.sin_w; pos = ww; idx = p - a.tab.pt - a.tab.ph; stride = a.tab.pw;
+              ct = tcw; stb = tsw; off = w_off + (p - a.tab.pt - a.tab.ph);
             }
-            if (valid) {
-              const float cs = __ldg(ct + (size_t)pos * stride + idx);
-              const float sn = __ldg(stb + (size_t)pos * stride + idx);
-              const float r0 = y0 * cs - y1 * sn;
-              y1 = y0 * sn + y1 * cs;
-              y0 = r0;
-            }
+            cs[i] = ct[off];
+            sn[i] = stb[off];
           }
-          pk[i] = valid ? cvt_bf16x2(y0, y1) : 0u;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float y0 = __uint_as_float(o[2 * i]), y1 = __uint_as_float(o[2 * i + 1]);
+            pk[i] = valid ? cvt_bf16x2(y0 * cs[i] - y1 * sn[i], y0 * sn[i] + y1 * cs[i]) : 0u;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = valid ? cvt_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])) : 0u;
         }
         if (in_chunk) {
           const size_t bh = (size_t)b * d.H + head;
@@ -260,6 +337,9 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
           }
         }
       }
+      // buffer u is read: the MMAs of the tile after next may overwrite it
+      tc_fence_before();
+      mbar_arrive(&bar[kQBarAccEmpty + u]);
     }
   }
 
@@ -267,7 +347,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
   __syncthreads();
   if (warp == kQkvMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kQkvBN);
+    tmem_dealloc(tmem, 2 * kQkvBN);
   }
 }
 
@@ -283,7 +363,11 @@ cudaError_t launch_qkv_rope(const QkvArgs& a, const void* x, const void* w, cuda
   cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        QkvSmem::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.NT, a.MT, d.B);
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    nsm = 148;
+  const int ntiles = a.NT * a.MT * d.B;
+  dim3 grid(ntiles < nsm ? ntiles : nsm);  // persistent: one CTA per SM
   qkv_rope_kernel<<<grid, kQkvThreads, QkvSmem::kAlloc, stream>>>(mx, mw, a);
   return cudaGetLastError();
 }

@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--stream", action="store_true",
                     help="streaming run: every chunk of the workload through all its layers, "
                          "per-chunk latency percentiles (measurement mode, not the bench line)")
+    ap.add_argument("--qkv", action="store_true",
+                    help="the QKV projection fused with rotation/append/pooling (hidden = H*D) "
+                         "against cuBLAS GEMMs followed by the separate kernels (measurement mode)")
     return ap.parse_args()
 
 
@@ -643,10 +646,77 @@ def run_stream(args):
     return 0
 
 
+def run_qkv(args):
+    """Fused QKV projection + rotation + append + pooling of one chunk, against
+    the unfused route on the same inputs: three cuBLAS GEMMs (q, k, v), then
+    cva_rope3d_apply + cva_hsa_compress for q and cva_kv_append for k, v.
+    Medians of --steps runs, L2 flushed before each."""
+    import numpy as np
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    from cva_workload import WORKLOADS, hidden_inputs
+    wl = WORKLOADS[args.workload]
+    C = wl.H * wl.D
+    inp = hidden_inputs(wl, C)
+    dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    shape = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
+    tables = ops.DeviceRopeTables(wl.D, wl.t0 + wl.Fc, wl.Fh, wl.Fw)
+    cache = ops.DeviceKVCache(shape, wl.window, 0)
+    q_rot = torch.empty((wl.B, wl.H, wl.Fc * wl.T_pad, wl.D), dtype=torch.bfloat16, device="cuda")
+    qpool = torch.empty((wl.B, wl.H, wl.NQB, wl.D), dtype=torch.float32, device="cuda")
+    HD = wl.H * wl.D
+    wq, wk, wv = w[:HD], w[HD:2 * HD], w[2 * HD:]
+    flush = L2Flush()
+
+    def fused():
+        ops.qkv_rope_append(x, w, cache, tables, wl.t0, q_rot, qpool)
+
+    def unfused():
+        q = torch.matmul(x, wq.t())
+        k = torch.matmul(x, wk.t())
+        v = torch.matmul(x, wv.t())
+        ops.rope3d_apply(q, q_rot, tables, shape, wl.t0, 1)
+        ops.hsa_compress(q_rot, shape, qpool)
+        ops.kv_append(k, v, cache, tables, wl.t0)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 1)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    f_ms = timed(fused)
+    u_ms = timed(unfused)
+    assert ops.device_status() == 0
+    flops = 2.0 * wl.B * wl.Lq * C * 3 * HD
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    print(json.dumps({
+        "mode": "qkv projection", "workload": wl.key, "hidden": C, "gemm": f"[{wl.B * wl.Lq} x {C}] x [{C} x {3 * HD}]",
+        "fused_us": 1e3 * f_ms, "fused_tflops": flops / (f_ms * 1e-3) / 1e12,
+        "fused_frac_of_bf16_peak": flops / (f_ms * 1e-3) / 1e12 / peak, "peak_source": f"{src} bf16 burst",
+        "unfused_us": 1e3 * u_ms, "speedup": u_ms / f_ms, "steps": args.steps, "stat": "median",
+        "launches": {"fused": 2, "unfused": 3 + 4}}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.qkv:
+        return run_qkv(args)
     if args.sweep:
         return run_sweep(args)
     if args.stream:
