@@ -44,9 +44,10 @@ constexpr int kQkvBM = 128;
 constexpr int kQkvBN = 256;
 constexpr int kQkvBK = 64;       // one 128-byte swizzle row of bf16
 constexpr int kQkvStages = 4;
-constexpr int kQkvThreads = 192;
-constexpr int kQkvProducerWarp = 4;
-constexpr int kQkvMmaWarp = 5;
+constexpr int kQkvEpiWarps = 8;   // two per TMEM lane quarter, each half of the columns
+constexpr int kQkvThreads = 32 * kQkvEpiWarps + 64;
+constexpr int kQkvProducerWarp = kQkvEpiWarps;
+constexpr int kQkvMmaWarp = kQkvEpiWarps + 1;
 constexpr int kQkvGroupM = 8;
 
 struct QkvSmem {
@@ -55,12 +56,12 @@ struct QkvSmem {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kA = 0;                         // stage s at + s * kStageBytes
   static constexpr int kB = kABytes;
-  static constexpr int kRed = kQkvStages * kStageBytes;  // [2][4 warps][32] column sums
-  static constexpr int kTab = kRed + 2 * 4 * 32 * 4;       // cos/sin tables of the chunk
+  static constexpr int kRed = kQkvStages * kStageBytes;  // [2 groups][2][4 warps][32] column sums
+  static constexpr int kTab = kRed + 2 * 2 * 4 * 32 * 4;   // cos/sin tables of the chunk
   static constexpr int kTabFloats = 7168;
   static constexpr int kBar = kTab + kTabFloats * 4;
   static constexpr int kMisc = kBar + 16 * 8;
-  static constexpr int kBytes = kMisc + 32;
+  static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory of one CTA");
 };
@@ -70,8 +71,11 @@ struct QkvSmem {
 constexpr int kQBarFull = 0, kQBarEmpty = kQkvStages, kQBarAccFull = 2 * kQkvStages,
               kQBarAccEmpty = 2 * kQkvStages + 2;
 
-__device__ __forceinline__ void qkv_epi_sync() {  // the 4 epilogue warps
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+__device__ __forceinline__ void qkv_epi_sync() {  // all epilogue warps
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kQkvEpiWarps) : "memory");
+}
+__device__ __forceinline__ void qkv_group_sync(int g) {  // the 4 warps of column half g
+  asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory");
 }
 
 __global__ void __launch_bounds__(kQkvThreads, 1)
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&bar[kQBarAccFull + u], 1);
-      mbar_init(&bar[kQBarAccEmpty + u], 128);
+      mbar_init(&bar[kQBarAccEmpty + u], 32 * kQkvEpiWarps);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -195,9 +199,11 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int r = tid;  // row of the tile = TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    volatile int* okw = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [4]
+    const int quarter = warp & 3;        // TMEM lane quarter
+    const int grp = warp >> 2;           // column half: chunks 4 grp .. 4 grp + 3
+    const int r = quarter * 32 + lane;   // row of the tile = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    volatile int* okw = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);  // [8]
     // While the MMAs run: copy the cos/sin rows the chunk needs into shared
     // memory: [cos_t, sin_t] of frames t0 .. t0+Fc-1, then [cos_h, sin_h]
     // (Fh rows), then [cos_w, sin_w] (Fw rows).
@@ -207,11 +213,12 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     if (stab) {
       const float* src_t = a.tab.cos_t + (size_t)a.t0 * a.tab.pt;
       const float* src_ts = a.tab.sin_t + (size_t)a.t0 * a.tab.pt;
-      for (int i = tid; i < nt_f; i += 128) { tb[i] = src_t[i]; tb[nt_f + i] = src_ts[i]; }
+      constexpr int kN = 32 * kQkvEpiWarps;
+      for (int i = tid; i < nt_f; i += kN) { tb[i] = src_t[i]; tb[nt_f + i] = src_ts[i]; }
       float* th = tb + 2 * nt_f;
-      for (int i = tid; i < nh_f; i += 128) { th[i] = a.tab.cos_h[i]; th[nh_f + i] = a.tab.sin_h[i]; }
+      for (int i = tid; i < nh_f; i += kN) { th[i] = a.tab.cos_h[i]; th[nh_f + i] = a.tab.sin_h[i]; }
       float* tw = th + 2 * nh_f;
-      for (int i = tid; i < nw_f; i += 128) { tw[i] = a.tab.cos_w[i]; tw[nw_f + i] = a.tab.sin_w[i]; }
+      for (int i = tid; i < nw_f; i += kN) { tw[i] = a.tab.cos_w[i]; tw[nw_f + i] = a.tab.sin_w[i]; }
     }
     qkv_epi_sync();
     for (int id = blockIdx.x, lt = 0; id < ntiles; id += gridDim.x, ++lt) {
@@ -221,8 +228,10 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       bool ok = mbar_wait(&bar[kQBarAccFull + u], (lt >> 1) & 1, abort_flag, a.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (lane == 0) okw[warp] = ok ? 1 : 0;
-      qkv_epi_sync();  // the four warps take the same path through the barriers below
-      ok = okw[0] && okw[1] && okw[2] && okw[3];
+      qkv_epi_sync();  // the epilogue warps take the same path through the barriers below
+      ok = true;
+#pragma unroll
+      for (int w = 0; w < kQkvEpiWarps; ++w) ok = ok && okw[w] != 0;
       qkv_epi_sync();  // okw is rewritten for the next tile
       if (!ok) break;
       tc_fence_after();
@@ -251,10 +260,10 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       const int jb = f * d.nb + j;               // query block of the chunk
       const float vcnt = (float)((j == d.nb - 1) ? d.tail : d.blk);
       const int wpb = d.blk / 32;                // warps per block
-      const int w0 = (warp / wpb) * wpb;         // first warp of this row's block
+      const int w0 = (quarter / wpb) * wpb;      // first lane quarter of this row's block
       const int HD = d.H * d.D;
-      float* red = reinterpret_cast<float*>(smem + L::kRed);
-      for (int cc = 0; cc < kQkvBN / 32; ++cc) {
+      float* red = reinterpret_cast<float*>(smem + L::kRed) + grp * 2 * 128;
+      for (int cc = 4 * grp; cc < 4 * grp + 4; ++cc) {
         const int c = nt * kQkvBN + 32 * cc;
         if (c >= 3 * HD) break;                  // uniform: the projection has 3HD outputs
         const int which = c / HD;                // 0 q, 1 k, 2 v
@@ -325,10 +334,10 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
             }
           }
           float* rb = red + (cc & 1) * 128;
-          rb[warp * 32 + lane] = v[0];
-          qkv_epi_sync();
+          rb[quarter * 32 + lane] = v[0];
+          qkv_group_sync(grp);
           const int prb = mt * kQkvBM + w0 * 32;   // first row of the block
-          if (warp == w0 && prb / d.T_pad < d.Fc) {
+          if (quarter == w0 && prb / d.T_pad < d.Fc) {
             float s = 0.f;
             for (int w = 0; w < wpb; ++w) s += rb[(w0 + w) * 32 + lane];
             const size_t bh = (size_t)b * d.H + head;
