@@ -73,6 +73,9 @@ _SIGS = {
     "cva_history_frames": (c_int32, [P(KVCache), c_int32, P(c_int32), P(c_int32)]),
     "cva_qkv_rope_append": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
                                       c_void_p, c_void_p, c_void_p]),
+    "cva_chunk_attention_qkv": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
+                                          c_int32, c_int32, c_void_p, ctypes.c_size_t, c_void_p, c_void_p,
+                                          c_void_p]),
     "cva_hsa_compress": (c_int32, [c_void_p, P(Shape), c_void_p, c_void_p, c_void_p]),
     "cva_hsa_select": (c_int32, [c_void_p, P(KVCache), c_int32, c_int32, c_int32, c_void_p,
                                  c_void_p, c_void_p, c_void_p]),
@@ -291,6 +294,16 @@ def qkv_rope_append(x, w_qkv, cache: DeviceKVCache, tables: DeviceRopeTables, t0
     check(lib.cva_qkv_rope_append(_ptr(x), _ptr(w_qkv), int(x.shape[-1]), ctypes.byref(cache.struct),
                                   ctypes.byref(tables.struct), t0, _ptr(q_rot), _ptr(qpool_blk),
                                   _stream(stream)))
+
+
+def chunk_attention_qkv(x, w_qkv, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, k_f: int,
+                        k_b: int, workspace, out, lse=None, stream=None) -> None:
+    """chunk_attention starting from the hidden states x [B, Lq, C] and the
+    fused projection weight w_qkv [3*H*D, C]."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib.cva_chunk_attention_qkv(_ptr(x), _ptr(w_qkv), int(x.shape[-1]), ctypes.byref(cache.struct),
+                                      ctypes.byref(tables.struct), t0, k_f, k_b, _ptr(workspace), ws_bytes,
+                                      _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def hsa_compress(q_rot, shape: Shape, qpool_blk, qpool_frm=None, stream=None) -> None:

@@ -581,6 +581,57 @@ int cva_blocksparse_attn_fwd(const void* q_rot, const cva_kv_cache* cache, int32
                    workspace, workspace ? ws_bytes : 0, static_cast<cudaStream_t>(stream));
 }
 
+int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, const cva_kv_cache* cache,
+                            const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                            void* workspace, size_t ws_bytes, void* out, float* lse, cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!out || !workspace) return fail(CVA_EINVAL, "NULL buffer");
+  if (!aligned(out, 16) || !aligned(workspace, 256))
+    return fail(CVA_EINVAL, "out must be 16-byte and workspace 256-byte aligned");
+  const Dims d = make_dims(cache->shape);
+  const bool dense = k_f < 0;
+  const ChunkWs w = chunk_ws_layout(d, dense ? 0 : k_f, dense ? 0 : k_b);
+  if (ws_bytes < w.total) return fail(CVA_ENOMEM, "workspace %zu bytes < %zu needed", ws_bytes, w.total);
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
+  if (!dense) {
+    const int kfe = k_f < F ? k_f : F;
+    if (F > 0 && k_f < 1) return fail(CVA_ERANGE, "k_f must be >= 1 when there is history");
+    if (k_b < 0 || (int64_t)k_b > (int64_t)kfe * d.nb)
+      return fail(CVA_ERANGE, "k_b %d outside [0, %d] (k_f_eff * blocks per frame)", k_b, kfe * d.nb);
+    if (F > 256) return fail(CVA_ENOTSUP, "history frames %d > 256", F);
+    if ((int64_t)kfe * d.nb > 1024) return fail(CVA_ENOTSUP, "candidate blocks %d > 1024", kfe * d.nb);
+  }
+  rc = check_attn_limits(d, F, dense || F == 0, dense ? 0 : k_b);
+  if (rc) return rc;
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws + w.q_rot);
+  float* qpool = reinterpret_cast<float*>(ws + w.qpool);
+  int32_t* fidx = reinterpret_cast<int32_t*>(ws + w.frame_idx);
+  int32_t* bidx = reinterpret_cast<int32_t*>(ws + w.block_idx);
+  int32_t* bcnt = reinterpret_cast<int32_t*>(ws + w.block_cnt);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool sparse = !dense && F > 0;
+  cudaError_t e = stage_mark(0, s);
+  if (e != cudaSuccess) return cuda_fail(e, "stage event");
+  // steps 1-3: projection, rotation, append and pooling in the fused kernel
+  rc = cva_qkv_rope_append(x, w_qkv, hidden, cache, tables, t0, q_rot, sparse ? qpool : nullptr, stream);
+  if (rc) return rc;
+  if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  if (sparse) {
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, s);
+    if (rc) return rc;
+  }
+  if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s);
+  if (rc) return rc;
+  if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  return CVA_OK;
+}
+
 int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, size_t* bytes) {
   int rc = check_shape(shape);
   if (rc) return rc;

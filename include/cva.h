@@ -269,6 +269,18 @@ int cva_chunk_attention(const void* q, const void* k, const void* v,
                         int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
                         size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
+/* Steps 1-5 for one chunk starting from the hidden states: the fused QKV
+ * projection with Causal-RoPE, append and pooling (cva_qkv_rope_append, the
+ * pages' section 2C operator fusion), then selection with (k_f, k_b)
+ * (dense when k_f < 0) and attention, all on the caller's stream.
+ *   x: bf16 [B, Lq, C]; w_qkv: bf16 [3*H*D, C] (as cva_qkv_rope_append);
+ *   out: bf16 [B, Lq, H, D]; lse: fp32 [B][H][Lq] or NULL;
+ *   workspace: cva_chunk_workspace_bytes() bytes (256-byte aligned). */
+int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden,
+                            const cva_kv_cache* cache, const cva_rope_tables* tables,
+                            int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
+                            size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
+
 /* The fused chunk call without a caller workspace (the pages have no
  * counterpart; this exists for callers that cannot allocate device memory
  * when they call, such as a plugin whose host runtime owns every allocation

@@ -121,3 +121,71 @@ def test_qkv_rope_append_rejects_bad_hidden():
     with pytest.raises(ops.CvaError):
         ops.qkv_rope_append(x, w, cache, tabs, wl.t0, q_rot)
     assert "multiple of 64" in ops.last_error()
+
+
+# ---- whole path from the hidden states ----------------------------------------------------
+
+def _oracle_stream_qkv(wl, hidden, w64, upto):
+    """Oracle over chunks 1..upto fed by the projection (one weight for the
+    layer): history appended as bf16 rotated k and bf16 v; returns the last
+    chunk's path intermediates (selection, rotated q) without attention."""
+    from _util import oracle_budget
+    cache = o_path.FrameCache(wl.B, wl.H, wl.D, wl.T_f, wl.blk, wl.window)
+    cache.t_begin = 0
+    for c in range(1, upto + 1):
+        x64 = bits_to_f64(hidden_inputs(wl, hidden, c)["x"])
+        q, k, v = o_qkv.project(x64, w64, wl.H, wl.D)
+        v = o_path.round_bf16(v)
+        t0 = wl.t0_of(c)
+        if c < upto:
+            _, k_rot = o_path.rotate_chunk(q, k, wl.Fh, wl.Fw, wl.Fc, t0, "bf16")
+            cache.append(k_rot, v, t0, wl.Fc)
+            continue
+        k_f, k_b = oracle_budget(wl, c)
+        run = o_path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0, k_f=k_f, k_b=k_b,
+                               dense=wl.dense, store="bf16", attend_too=False)
+        run.update(cache=cache, t0=t0)
+        return run
+
+
+@pytest.mark.parametrize("key,hidden", [("c1", 128), ("c1s", 64), ("r64", 192), ("r128", 256), ("r64s", 128)])
+def test_chunk_attention_from_hidden_states(key, hidden):
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    from _util import MAX_ABS, MEAN_ABS, attn_errors, lib_budget
+
+    wl = WORKLOADS[key]
+    upto = wl.chunk
+    w_bits = hidden_inputs(wl, hidden, 1)["w"]      # one weight for the layer
+    w64 = bits_to_f64(w_bits)
+    shp = shape_of(wl)
+    tabs = ops.DeviceRopeTables(wl.D, wl.t0_of(upto) + wl.Fc, wl.Fh, wl.Fw)
+    cache = ops.DeviceKVCache(shp, wl.window, 0)
+    wd = to_dev(w_bits)
+    for c in range(1, upto + 1):
+        k_f, k_b = (-1, 0) if wl.dense else lib_budget(wl, c)
+        ws = torch.empty(ops.chunk_workspace_bytes(shp, k_f, k_b), dtype=torch.uint8, device="cuda")
+        out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+        ops.chunk_attention_qkv(to_dev(hidden_inputs(wl, hidden, c)["x"]), wd, cache, tabs, wl.t0_of(c),
+                                k_f, k_b, ws, out)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+
+    run = _oracle_stream_qkv(wl, hidden, w64, upto)
+    o_want, _ = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, run["blocks"])
+    got = bits_to_f64(from_dev(out))
+    g, w = got, o_want
+    if run["blocks"] is not None and k_b > 0:
+        # query blocks whose selection differs from the oracle's (near ties) are left out
+        bhq = wl.B * wl.H * wl.NQB
+        r256 = lambda n: (n + 255) // 256 * 256
+        off = r256(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r256(bhq * wl.D * 4) + r256(bhq * max(k_f, 0) * 4)
+        gb = ws[off:off + bhq * k_b * 4].cpu().numpy().view(np.int32).reshape(wl.B, wl.H, wl.NQB, k_b)
+        ok = np.all(gb == run["blocks"], axis=-1)
+        assert ok.mean() >= 0.98, ok.mean()
+        sel = np.arange(wl.Lq)
+        qb = (sel // wl.T_f) * wl.nb + (sel % wl.T_f) // wl.blk
+        mask = np.transpose(ok[:, :, qb], (0, 2, 1))[..., None]
+        g, w = np.where(mask, g, 0.0), np.where(mask, w, 0.0)
+    mx, mean, rel = attn_errors(g, w)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
