@@ -143,3 +143,63 @@ def budget(chunk: int, hist_frames: int, nb: int, *, dense: bool, k_f_max: int,
     d = density(d_base, d_slope, d_pivot, chunk)
     k_b = math.floor(d * all_blocks + Fraction(1, 2))
     return k_f, min(cand, k_b)
+
+
+# --- chunk budget from the noise level (Light Forcing section 2.1) -------------------
+
+NOISE_BISECTION_STEPS = 200
+
+
+def noise_densities(n_chunks: int, Fc: int, window: int, nb: int, s_base: float, s_target: float):
+    """Key density of chunks 2..n from ``s_i = s_base - alpha_i * beta``.
+
+    Light Forcing, section 2.1: ``alpha_i`` scales with the noise level as
+    ``1/sqrt(T)`` and ``beta`` is set so that the total attention FLOPs meet
+    a target sparsity. Readings (the pages garble the formula):
+
+    * the noise level of chunk ``i`` grows with its index in the chunk
+      schedule, ``alpha_i = 1 / sqrt(i)``, so later chunks get more sparsity;
+    * density is ``d_i = 1 - s_i``, clamped to [0, 1], and counts history
+      blocks (the current chunk is always dense);
+    * the FLOP target is ``sum_i d_i N_i = (1 - s_target) sum_i N_i`` over
+      chunks 2..n, with ``N_i`` the history blocks of chunk ``i`` in a
+      rolling window of ``window`` frames;
+    * ``beta`` is found by bisection on [-2^20, 2^20] (the sum grows with
+      beta) in a fixed number of fp64 steps, the same in the library.
+
+    Returns ``{i: d_i}`` for i = 2..n (chunk 1 is dense).
+    """
+    chunks = list(range(2, n_chunks + 1))
+    N = {i: min(Fc * (i - 1), window - Fc) * nb for i in chunks}
+    alpha = {i: 1.0 / math.sqrt(i) for i in chunks}
+    d0 = 1.0 - s_base
+    goal = (1.0 - s_target) * sum(N[i] for i in chunks)
+
+    def dens(i, beta):
+        return min(max(d0 + alpha[i] * beta, 0.0), 1.0)
+
+    def total(beta):
+        s = 0.0
+        for i in chunks:
+            s += dens(i, beta) * N[i]
+        return s
+
+    lo, hi = -1048576.0, 1048576.0
+    for _ in range(NOISE_BISECTION_STEPS):
+        mid = 0.5 * (lo + hi)
+        if total(mid) < goal:
+            lo = mid
+        else:
+            hi = mid
+    return {i: dens(i, hi) for i in chunks}
+
+
+def noise_budget(chunk: int, hist_frames: int, nb: int, k_f_max: int, density_i: float) -> Tuple[int, int]:
+    """``(k_f, k_b)`` of a chunk with a given density: ``k_f = min(k_f_max,
+    history)`` and ``k_b = floor(d * history blocks + 1/2)`` at most the
+    candidates ``k_f * nb`` (as :func:`budget`, in fp64 for the density)."""
+    all_blocks = hist_frames * nb
+    if chunk <= 1 or hist_frames == 0:
+        return hist_frames, all_blocks
+    k_f = min(k_f_max, hist_frames)
+    return k_f, min(k_f * nb, int(math.floor(density_i * all_blocks + 0.5)))

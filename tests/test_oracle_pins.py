@@ -423,3 +423,48 @@ def test_qkv_rotation_after_projection_keeps_pair_norms_of_the_projection():
     np.testing.assert_allclose(n(kr), n(k), rtol=1e-12)
     np.testing.assert_array_equal(vv, v)
     assert not np.allclose(qr, q)
+
+
+# ---- CAG from the noise level ---------------------------------------------------------
+
+def test_noise_schedule_equal_targets_give_the_base_density():
+    # s_target = s_base: beta = 0, every chunk at density 1 - s_base
+    d = hsa.noise_densities(10, 3, 21, 25, 0.75, 0.75)
+    assert all(abs(v - 0.25) < 1e-12 for v in d.values())
+
+
+def test_noise_schedule_meets_the_flop_target_and_decreases():
+    # unclamped: sum d_i N_i = (1 - s_target) sum N_i; alpha_i = i^-1/2 makes
+    # later chunks sparser; the closed form beta = (s_base - s_target) sum N / sum alpha N
+    n, Fc, W, nb, sb, st = 12, 3, 21, 25, 0.9, 0.8
+    d = hsa.noise_densities(n, Fc, W, nb, sb, st)
+    N = {i: min(Fc * (i - 1), W - Fc) * nb for i in d}
+    tot = sum(d[i] * N[i] for i in d)
+    assert abs(tot - (1 - st) * sum(N.values())) < 1e-9 * sum(N.values())
+    vals = [d[i] for i in sorted(d)]
+    assert all(a > b for a, b in zip(vals, vals[1:]))
+    beta = (sb - st) * sum(N.values()) / sum(N[i] / math.sqrt(i) for i in N)
+    for i in d:
+        assert abs(d[i] - ((1 - sb) + beta / math.sqrt(i))) < 1e-9
+
+
+def test_noise_schedule_clamps_at_full_density():
+    # a target denser than the base can give pushes early chunks to density 1
+    d = hsa.noise_densities(6, 3, 60, 25, 0.5, 0.05)
+    assert max(d.values()) == 1.0 and min(d.values()) < 1.0
+    N = {i: min(3 * (i - 1), 57) * 25 for i in d}
+    assert abs(sum(d[i] * N[i] for i in d) - 0.95 * sum(N.values())) < 1e-6 * sum(N.values())
+
+
+def test_noise_budget_rounding_and_cap():
+    assert hsa.noise_budget(1, 0, 25, 8, 0.3) == (0, 0)
+    assert hsa.noise_budget(3, 6, 25, 8, 0.3) == (6, 45)        # 0.3 * 150 = 45
+    assert hsa.noise_budget(3, 6, 25, 2, 0.9) == (2, 50)        # capped at 2 * 25
+    assert hsa.noise_budget(2, 3, 25, 8, 0.19) == (3, 14)       # 14.25 -> 14
+
+
+def test_noise_schedule_sparser_target_makes_early_chunks_sparser_first():
+    # a target sparser than the base: beta < 0, early chunks lose the most
+    d = hsa.noise_densities(8, 3, 21, 25, 0.7, 0.8)
+    vals = [d[i] for i in sorted(d)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
