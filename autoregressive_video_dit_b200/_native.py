@@ -73,6 +73,10 @@ _SIGS = {
     "cva_history_frames": (c_int32, [P(KVCache), c_int32, P(c_int32), P(c_int32)]),
     "cva_qkv_rope_append": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
                                       c_void_p, c_void_p, c_void_p]),
+    "cva_cag_noise_densities": (c_int32, [c_int32, c_int32, c_int32, c_int32, ctypes.c_double,
+                                          ctypes.c_double, c_void_p]),
+    "cva_cag_density_budget": (c_int32, [c_int32, c_int32, c_int32, c_int32, ctypes.c_double, P(c_int32),
+                                         P(c_int32)]),
     "cva_chunk_attention_qkv": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
                                           c_int32, c_int32, c_void_p, ctypes.c_size_t, c_void_p, c_void_p,
                                           c_void_p]),
@@ -304,6 +308,22 @@ def chunk_attention_qkv(x, w_qkv, cache: DeviceKVCache, tables: DeviceRopeTables
     check(lib.cva_chunk_attention_qkv(_ptr(x), _ptr(w_qkv), int(x.shape[-1]), ctypes.byref(cache.struct),
                                       ctypes.byref(tables.struct), t0, k_f, k_b, _ptr(workspace), ws_bytes,
                                       _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def cag_noise_densities(n_chunks: int, Fc: int, window: int, blocks_per_frame: int, s_base: float,
+                        s_target: float) -> dict:
+    """{chunk: density} for chunks 2..n_chunks (see cva.h)."""
+    buf = (ctypes.c_double * (n_chunks - 1))()
+    check(lib.cva_cag_noise_densities(n_chunks, Fc, window, blocks_per_frame, s_base, s_target, buf))
+    return {i + 2: buf[i] for i in range(n_chunks - 1)}
+
+
+def cag_density_budget(chunk: int, hist_frames: int, blocks_per_frame: int, k_f_max: int,
+                       density: float) -> Tuple[int, int]:
+    kf, kb = c_int32(), c_int32()
+    check(lib.cva_cag_density_budget(chunk, hist_frames, blocks_per_frame, k_f_max, density,
+                                     ctypes.byref(kf), ctypes.byref(kb)))
+    return kf.value, kb.value
 
 
 def hsa_compress(q_rot, shape: Shape, qpool_blk, qpool_frm=None, stream=None) -> None:

@@ -23,7 +23,7 @@ LIB = os.path.join(PKG, "libcva.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr",
-              "-Xcompiler", "-fPIC,-O3", "-I", INCLUDE, "-I", CSRC] + ARCH
+              "-Xcompiler", "-fPIC,-O3,-ffp-contract=off", "-I", INCLUDE, "-I", CSRC] + ARCH
 
 
 def nvcc() -> str:

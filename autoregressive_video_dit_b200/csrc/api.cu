@@ -632,6 +632,62 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   return CVA_OK;
 }
 
+int cva_cag_noise_densities(int32_t n_chunks, int32_t Fc, int32_t window, int32_t blocks_per_frame,
+                            double s_base, double s_target, double* densities) {
+  if (!densities) return fail(CVA_EINVAL, "densities is NULL");
+  if (n_chunks < 2 || Fc < 1 || window < Fc || blocks_per_frame < 1)
+    return fail(CVA_EINVAL, "n_chunks >= 2, Fc >= 1, window >= Fc and blocks_per_frame >= 1 required");
+  if (!(s_base >= 0.0 && s_base <= 1.0 && s_target >= 0.0 && s_target <= 1.0))
+    return fail(CVA_EINVAL, "sparsities must lie in [0, 1]");
+  // Same fp64 operations, in the same order, as the reference statement.
+  const int n = n_chunks - 1;  // chunks 2..n_chunks
+  auto N = [&](int i) { int f = Fc * (i - 1); if (f > window - Fc) f = window - Fc; return (double)f * blocks_per_frame; };
+  auto alpha = [&](int i) { return 1.0 / sqrt((double)i); };
+  const double d0 = 1.0 - s_base;
+  double nsum = 0.0;
+  for (int i = 2; i <= n_chunks; ++i) nsum += N(i);
+  const double goal = (1.0 - s_target) * nsum;
+  auto dens = [&](int i, double beta) {
+    double v = d0 + alpha(i) * beta;
+    if (v < 0.0) v = 0.0;
+    if (v > 1.0) v = 1.0;
+    return v;
+  };
+  auto total = [&](double beta) {
+    double s = 0.0;
+    for (int i = 2; i <= n_chunks; ++i) s += dens(i, beta) * N(i);
+    return s;
+  };
+  double lo = -1048576.0, hi = 1048576.0;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (total(mid) < goal) lo = mid;
+    else hi = mid;
+  }
+  for (int k = 0; k < n; ++k) densities[k] = dens(k + 2, hi);
+  return CVA_OK;
+}
+
+int cva_cag_density_budget(int32_t chunk_index, int32_t hist_frames, int32_t blocks_per_frame,
+                           int32_t k_f_max, double density, int32_t* k_f, int32_t* k_b) {
+  if (!k_f || !k_b) return fail(CVA_EINVAL, "k_f or k_b is NULL");
+  if (hist_frames < 0 || blocks_per_frame < 1 || k_f_max < 0 || !(density >= 0.0 && density <= 1.0))
+    return fail(CVA_EINVAL, "bad budget arguments");
+  const int64_t all = (int64_t)hist_frames * blocks_per_frame;
+  if (chunk_index <= 1 || hist_frames == 0) {
+    *k_f = hist_frames;
+    *k_b = (int32_t)all;
+    return CVA_OK;
+  }
+  const int kf = k_f_max < hist_frames ? k_f_max : hist_frames;
+  int64_t kb = (int64_t)floor(density * (double)all + 0.5);
+  const int64_t cand = (int64_t)kf * blocks_per_frame;
+  if (kb > cand) kb = cand;
+  *k_f = kf;
+  *k_b = (int32_t)kb;
+  return CVA_OK;
+}
+
 int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, size_t* bytes) {
   int rc = check_shape(shape);
   if (rc) return rc;

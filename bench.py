@@ -552,9 +552,17 @@ def run_sweep(args):
     base = WORKLOADS[args.workload]
     stream = torch.cuda.current_stream()
     flush = L2Flush()
-    for sched, slope in (("literal", base.d_slope), ("mirrored", -base.d_slope)):
+    # third schedule: density from the noise level (s_base 0.8, target 0.75)
+    noise = ops.cag_noise_densities(base.chunks, base.Fc, base.window, base.nb, 0.8, 0.75)
+    schedules = [("literal", base.d_slope, None), ("mirrored", -base.d_slope, None),
+                 ("noise s_base=0.8 s_target=0.75", base.d_slope, noise)]
+    for sched, slope, dens in schedules:
         for chunk in range(1, base.chunks + 1):
             wl = base.replace(d_slope=slope).with_chunk(chunk)
+            if dens is not None and chunk >= 2:
+                hist = min(base.Fc * (chunk - 1), base.window - base.Fc)
+                _, kb = ops.cag_density_budget(chunk, hist, base.nb, base.k_f_max, dens[chunk])
+                wl = wl.replace(k_b_fixed=kb)
             st = setup_workload(args, layer=0, wl=wl)
 
             def step():

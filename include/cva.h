@@ -314,6 +314,23 @@ int cva_set_stage_events(void* const* events, int32_t n);
  * n floats. Not used by the path itself; it lets tests bound the error. */
 int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream);
 
+/* Chunk budget from the noise level ("Light Forcing", section 2.1: s_i =
+ * s_base - alpha_i beta, alpha_i scaling with the noise level as 1/sqrt(T),
+ * beta set so that the total FLOPs meet a target sparsity). Readings: alpha_i
+ * = 1/sqrt(i) for chunk i (the noise level grows with the chunk index);
+ * density d_i = 1 - s_i clamped to [0, 1] over history blocks; the target is
+ * sum_i d_i N_i = (1 - s_target) sum_i N_i over chunks 2..n_chunks, N_i the
+ * history blocks of chunk i in a rolling window of `window` frames (chunks
+ * of Fc frames, blocks_per_frame blocks); beta by 200 fp64 bisection steps on
+ * [-2^20, 2^20]. Writes densities[i - 2] for i = 2..n_chunks (chunk 1 is
+ * dense). CVA_EINVAL for n_chunks < 2, Fc < 1, window < Fc, or s outside [0, 1]. */
+int cva_cag_noise_densities(int32_t n_chunks, int32_t Fc, int32_t window, int32_t blocks_per_frame,
+                            double s_base, double s_target, double* densities);
+/* (k_f, k_b) of a chunk at a given density: k_f = min(k_f_max, history),
+ * k_b = floor(density * history blocks + 1/2) capped at k_f * blocks. */
+int cva_cag_density_budget(int32_t chunk_index, int32_t hist_frames, int32_t blocks_per_frame,
+                           int32_t k_f_max, double density, int32_t* k_f, int32_t* k_b);
+
 /* ---- cache arena ---------------------------------------------------------- */
 
 /* Bytes of one layer's cache for `window` frame slots (256-byte aligned parts). */

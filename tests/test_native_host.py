@@ -171,3 +171,25 @@ def test_workspace_bytes(ops):
             + r(bhq * 120 * 4) + r(bhq * 4) + attn)
     assert ops.chunk_workspace_bytes(s, 8, 120) == want
     assert ops.attn_workspace_bytes(s, 120) == attn
+
+
+@pytest.mark.parametrize("n,Fc,W,nb,sb,st", [(10, 3, 21, 25, 0.75, 0.7), (80, 3, 60, 25, 0.9, 0.8),
+                                              (7, 3, 21, 29, 0.8, 0.8), (6, 3, 60, 25, 0.5, 0.05),
+                                              (8, 3, 21, 25, 0.7, 0.8), (30, 2, 9, 3, 1.0, 0.6)])
+def test_noise_schedule_matches_oracle(ops, n, Fc, W, nb, sb, st):
+    want = o_hsa.noise_densities(n, Fc, W, nb, sb, st)
+    got = ops.cag_noise_densities(n, Fc, W, nb, sb, st)
+    assert got.keys() == want.keys()
+    for i in want:
+        assert got[i] == want[i], (i, got[i], want[i])     # same fp64 steps, same values
+        hist = min(Fc * (i - 1), W - Fc)
+        assert ops.cag_density_budget(i, hist, nb, 8, got[i]) == o_hsa.noise_budget(i, hist, nb, 8, want[i])
+
+
+def test_noise_schedule_rejects_bad_arguments(ops):
+    with pytest.raises(ops.CvaError):
+        ops.cag_noise_densities(1, 3, 21, 25, 0.75, 0.7)
+    with pytest.raises(ops.CvaError):
+        ops.cag_noise_densities(5, 3, 2, 25, 0.75, 0.7)
+    with pytest.raises(ops.CvaError):
+        ops.cag_noise_densities(5, 3, 21, 25, 1.5, 0.7)
