@@ -110,6 +110,53 @@ def block_select(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.ndarray
     return cand_ids[pos], gap
 
 
+def block_select_topp(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.ndarray,
+                      nb: int, T_f: int, blk: int, p: float, k_cap: int):
+    """Second level with a top-p budget instead of a fixed ``k_b``.
+
+    "Sparse VideoGen2", section B (centroid top-p): clusters are sorted by
+    their estimated attention scores and taken one after another until the
+    cumulative score reaches the threshold ``p``. Readings for key blocks:
+
+    * the candidates are the blocks of the picked frames, ranked as in
+      :func:`block_select` (pooled score ``q.kb``, ties to the lower
+      position);
+    * a block's estimated attention is its share of the softmax of the
+      pooled scores weighted by its valid token count,
+      ``m_c = n_c exp(s_c / sqrt(D)) / sum_c' n_c' exp(s_c' / sqrt(D))``;
+    * the shortest prefix of the ranking whose mass reaches ``p`` is taken:
+      block c goes in when the mass ranked above it is below ``p``; at least
+      one block, at most ``k_cap`` (the list size).
+
+    Returns the chosen ids ``t * nb + j`` (ascending) and a boundary gap: the
+    smallest of the relative score gap at the cut and the distance of the
+    threshold from the cumulative masses around the cut (``inf`` when no
+    candidate was left out).
+    """
+    frames_t = np.asarray(frames_t)
+    qbar = np.asarray(qbar, dtype=np.float64)
+    D = qbar.shape[0]
+    s = kbar_blocks.reshape(-1, kbar_blocks.shape[-1]) @ qbar
+    C = s.shape[0]
+    cand_ids = (frames_t[:, None] * nb + np.arange(nb)[None, :]).reshape(-1)
+    tail = T_f - (nb - 1) * blk
+    n = np.tile(np.array([blk] * (nb - 1) + [tail], dtype=np.float64), frames_t.shape[0])
+    order = np.lexsort((np.arange(C), -s))
+    m = n * np.exp((s - s.max()) / math.sqrt(D))
+    total = m.sum()
+    ms = m[order]
+    before = np.cumsum(ms) - ms                            # mass ranked above each candidate
+    take = (before < p * total) & (np.arange(C) < k_cap)
+    take[0] = k_cap > 0                                    # at least one block
+    r = int(take.sum())
+    gap = math.inf
+    if r < C:
+        gap = min(rel_gap(s[order[r - 1]], s[order[r]]) if r > 0 else math.inf,
+                  abs(before[r] - p * total) / total,
+                  abs(before[r - 1] - p * total) / total if r > 0 else math.inf)
+    return np.sort(cand_ids[order[:r]]), gap
+
+
 # --- chunk budget -----------------------------------------------------------------
 
 def density(d_base: Fraction, d_slope: Fraction, d_pivot: int, chunk: int) -> Fraction:

@@ -98,19 +98,21 @@ def pool_queries(q_rot: np.ndarray, T_f: int, blk: int, Fc: int):
 
 
 def select_chunk(qbar_blk: np.ndarray, cache: FrameCache, hist_t: np.ndarray,
-                 k_f: int, k_b: int):
+                 k_f: int, k_b: int, topp: Optional[float] = None):
     """Two-level selection for every (b, h, query block).
 
     Returns ``frames [B,H,NQB,k_f_eff]``, ``blocks [B,H,NQB,k_b]`` (ids
     ``t*nb + j``, ascending) and the relative boundary gaps ``gap_f``,
-    ``gap_b`` ``[B,H,NQB]`` (``inf`` where nothing was cut).
+    ``gap_b`` ``[B,H,NQB]`` (``inf`` where nothing was cut). With ``topp``
+    the second level is :func:`oracle.hsa.block_select_topp` with cap
+    ``k_b``: each row holds its chosen ids first, then ``-1``.
     """
     B, H, NQB, D = qbar_blk.shape
     nb = cache.nb
     F = hist_t.shape[0]
     k_f_eff = min(k_f, F)
     frames = np.zeros((B, H, NQB, k_f_eff), dtype=np.int64)
-    blocks = np.zeros((B, H, NQB, k_b), dtype=np.int64)
+    blocks = np.full((B, H, NQB, k_b), -1 if topp is not None else 0, dtype=np.int64)
     gap_f = np.full((B, H, NQB), math.inf)
     gap_b = np.full((B, H, NQB), math.inf)
     if F:
@@ -123,9 +125,13 @@ def select_chunk(qbar_blk: np.ndarray, cache: FrameCache, hist_t: np.ndarray,
                     continue
                 ft, gf = _hsa.frame_select(qbar_blk[b, h, qb], kf_all[b, h], hist_t, k_f)
                 pos = np.searchsorted(hist_t, ft)
-                ids, gb = _hsa.block_select(qbar_blk[b, h, qb], kb_all[b, h][pos], ft, nb, k_b)
+                if topp is None:
+                    ids, gb = _hsa.block_select(qbar_blk[b, h, qb], kb_all[b, h][pos], ft, nb, k_b)
+                else:
+                    ids, gb = _hsa.block_select_topp(qbar_blk[b, h, qb], kb_all[b, h][pos], ft, nb,
+                                                     cache.T_f, cache.blk, topp, k_b)
                 frames[b, h, qb] = ft
-                blocks[b, h, qb] = ids
+                blocks[b, h, qb, :len(ids)] = ids
                 gap_f[b, h, qb] = gf
                 gap_b[b, h, qb] = gb
     return frames, blocks, gap_f, gap_b
@@ -135,13 +141,16 @@ def keys_of_query_block(cache: FrameCache, b: int, h: int, t0: int, Fc: int,
                         block_ids: Optional[np.ndarray]):
     """K and V rows a query block attends to: the valid tokens of its picked
     history blocks (all history blocks when ``block_ids`` is None) followed by
-    every token of the current chunk's frames."""
+    every token of the current chunk's frames. Negative ids (list padding)
+    are skipped."""
     nb, blk, T_f = cache.nb, cache.blk, cache.T_f
     ks, vs = [], []
     if block_ids is None:
         hist = cache.history(t0, Fc)
         block_ids = (hist[:, None] * nb + np.arange(nb)[None, :]).reshape(-1)
     for g in np.asarray(block_ids):
+        if g < 0:
+            continue
         t, j = divmod(int(g), nb)
         fr = cache.frames[t]
         lo, hi = j * blk, min((j + 1) * blk, T_f)
@@ -193,11 +202,13 @@ def rotate_chunk(q: np.ndarray, k: np.ndarray, Fh: int, Fw: int, Fc: int, t0: in
 
 def run_chunk(cache: FrameCache, q: np.ndarray, k: np.ndarray, v: np.ndarray, *,
               Fh: int, Fw: int, Fc: int, t0: int, k_f: int, k_b: int,
-              dense: bool, store: str = "bf16", rows=None, attend_too: bool = True):
+              dense: bool, store: str = "bf16", rows=None, attend_too: bool = True,
+              topp: Optional[float] = None):
     """One chunk through the whole path; returns every intermediate.
 
     ``q, k, v`` are the raw ``[B, Lq, H, D]`` inputs (fp64 values). The cache
-    is updated in place.
+    is updated in place. ``topp`` switches the second selection level to the
+    top-p budget with cap ``k_b``.
     """
     q_rot, k_rot = rotate_chunk(q, k, Fh, Fw, Fc, t0, store)
     cache.append(k_rot, np.asarray(v, dtype=np.float64), t0, Fc)
@@ -209,7 +220,7 @@ def run_chunk(cache: FrameCache, q: np.ndarray, k: np.ndarray, v: np.ndarray, *,
         out.update(frames=None, blocks=None, gap_f=None, gap_b=None)
         blocks = None
     else:
-        frames, blocks, gf, gb = select_chunk(qbar_blk, cache, hist, k_f, k_b)
+        frames, blocks, gf, gb = select_chunk(qbar_blk, cache, hist, k_f, k_b, topp)
         out.update(frames=frames, blocks=blocks, gap_f=gf, gap_b=gb)
     if attend_too:
         o, lse = attend_chunk(q_rot, cache, t0, Fc, blocks, rows)

@@ -214,7 +214,7 @@ def test_frame_select_takes_all_when_few():
     assert list(ft) == [0, 1, 2] and gap == math.inf
 
 
-def _c1_path(wl, t_shift=0, store="bf16", dense=None):
+def _c1_path(wl, t_shift=0, store="bf16", dense=None, topp=None):
     """Run the c1 workload's chunks 1..4 through the oracle path."""
     cache = path.FrameCache(wl.B, wl.H, wl.D, wl.T_f, wl.blk, wl.window)
     out = None
@@ -228,7 +228,7 @@ def _c1_path(wl, t_shift=0, store="bf16", dense=None):
                               d_base=wl.d_base, d_slope=wl.d_slope, d_pivot=wl.d_pivot)
         out = path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0,
                              k_f=k_f, k_b=k_b, dense=wl.dense if dense is None else dense,
-                             store=store)
+                             store=store, topp=topp)
     return cache, out
 
 
@@ -468,3 +468,87 @@ def test_noise_schedule_sparser_target_makes_early_chunks_sparser_first():
     d = hsa.noise_densities(8, 3, 21, 25, 0.7, 0.8)
     vals = [d[i] for i in sorted(d)]
     assert all(a < b for a, b in zip(vals, vals[1:]))
+
+
+# ---- top-p block budget (SVG2 centroid top-p) ----------------------------------------
+
+def _topp_inputs(seed, F=3, nb=4, D=8):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal(D), rng.standard_normal((F, nb, D)), np.array([2, 5, 7, 9][:F])
+
+
+def test_topp_full_threshold_takes_everything_up_to_the_cap():
+    q, kb, ft = _topp_inputs(1)
+    ids, _ = hsa.block_select_topp(q, kb, ft, 4, 16, 5, 1.0 + 1e-12, 12)
+    assert len(ids) == 12
+    ids, _ = hsa.block_select_topp(q, kb, ft, 4, 16, 5, 1.0 + 1e-12, 5)
+    want, _ = hsa.block_select(q, kb, ft, 4, 5)                 # the cap is a top-k
+    np.testing.assert_array_equal(ids, want)
+
+
+def test_topp_tiny_threshold_takes_the_top_block():
+    q, kb, ft = _topp_inputs(2)
+    ids, _ = hsa.block_select_topp(q, kb, ft, 4, 16, 5, 1e-9, 12)
+    want, _ = hsa.block_select(q, kb, ft, 4, 1)
+    np.testing.assert_array_equal(ids, want)
+
+
+def test_topp_equal_scores_and_sizes_take_ceil_p_c():
+    # equal masses: the prefix before candidate r holds r/C of the mass
+    D, F, nb = 4, 2, 5
+    q = np.zeros(D)
+    kb = np.ones((F, nb, D))
+    ft = np.array([0, 1])
+    for p in (0.1, 0.25, 0.5, 0.61, 0.9):
+        ids, _ = hsa.block_select_topp(q, kb, ft, nb, nb * 8, 8, p, F * nb)
+        assert len(ids) == math.ceil(p * F * nb - 1e-12), (p, len(ids))
+        np.testing.assert_array_equal(ids, np.arange(len(ids)))   # ties: lower positions
+
+
+def test_topp_brute_force_shortest_prefix():
+    # the chosen set is the shortest prefix of the ranking whose size-weighted
+    # softmax mass reaches p (brute force over prefix lengths, written out)
+    for seed in range(20):
+        q, kb, ft = _topp_inputs(100 + seed, F=2, nb=3, D=6)
+        T_f, blk, nb = 11, 4, 3                                     # tail block of 3 tokens
+        s = kb.reshape(-1, 6) @ q
+        n = np.array([4, 4, 3, 4, 4, 3], dtype=float)
+        w = n * np.exp(s / math.sqrt(6))
+        order = sorted(range(6), key=lambda c: (-s[c], c))
+        p = 0.3 + 0.05 * (seed % 10)
+        best = None
+        for L in range(1, 7):
+            if sum(w[c] for c in order[:L]) >= p * w.sum():
+                best = L
+                break
+        ids, _ = hsa.block_select_topp(q, kb, ft, nb, T_f, blk, p, 6)
+        want = np.sort(np.array([ft[c // 3] * 3 + c % 3 for c in order[:best]]))
+        np.testing.assert_array_equal(ids, want)
+
+
+def test_topp_path_full_threshold_equals_dense():
+    # p just above 1 with the cap at every candidate keeps every history block
+    wl = WORKLOADS["c1s"].replace(k_f_max=9, k_b_fixed=9)
+    _, out = _c1_path(wl, topp=1.0 + 1e-9)
+    assert np.all(out["blocks"] >= 0)
+    _, outd = _c1_path(WORKLOADS["c1"])
+    np.testing.assert_allclose(outd["o"], out["o"], rtol=1e-12, atol=1e-13)
+
+
+def test_topp_path_rows_are_top_k_of_their_own_count():
+    # a top-p row with r blocks is the top-r of the candidates, -1 after them
+    wl = WORKLOADS["c1s"].replace(k_f_max=6, k_b_fixed=6)
+    cache, out = _c1_path(wl, topp=0.5)
+    cap = out["blocks"].shape[-1]
+    counts = (out["blocks"] >= 0).sum(-1)
+    assert counts.min() >= 1 and counts.max() <= cap and counts.min() < cap
+    for b in range(wl.B):
+        for h in range(wl.H):
+            for qb in range(wl.NQB):
+                row = out["blocks"][b, h, qb]
+                r = counts[b, h, qb]
+                assert np.all(row[r:] == -1)
+                ft = out["frames"][b, h, qb]
+                kb = np.stack([cache.frames[t]["kb"][b, h] for t in ft])
+                want, _ = hsa.block_select(out["qbar_blk"][b, h, qb], kb, ft, wl.nb, r)
+                np.testing.assert_array_equal(row[:r], want)
