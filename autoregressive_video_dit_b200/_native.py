@@ -83,6 +83,8 @@ _SIGS = {
     "cva_hsa_compress": (c_int32, [c_void_p, P(Shape), c_void_p, c_void_p, c_void_p]),
     "cva_hsa_select": (c_int32, [c_void_p, P(KVCache), c_int32, c_int32, c_int32, c_void_p,
                                  c_void_p, c_void_p, c_void_p]),
+    "cva_hsa_select_topp": (c_int32, [c_void_p, P(KVCache), c_int32, c_int32, c_int32, ctypes.c_float,
+                                      c_void_p, c_void_p, c_void_p, c_void_p]),
     "cva_attn_workspace_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
     "cva_blocksparse_attn_fwd": (c_int32, [c_void_p, P(KVCache), c_int32, c_void_p, c_void_p,
                                            c_int32, c_void_p, c_void_p, c_void_p, c_size_t,
@@ -91,6 +93,9 @@ _SIGS = {
     "cva_chunk_attention": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
                                       c_int32, c_int32, c_int32, c_void_p, c_size_t, c_void_p,
                                       c_void_p, c_void_p]),
+    "cva_chunk_attention_topp": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
+                                           c_int32, c_int32, c_int32, ctypes.c_float, c_void_p, c_size_t,
+                                           c_void_p, c_void_p, c_void_p]),
     "cva_chunk_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
                                               c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
@@ -337,6 +342,13 @@ def hsa_select(qpool_blk, cache: DeviceKVCache, t0: int, k_f: int, k_b: int, fra
                              _ptr(frame_idx), _ptr(block_idx), _ptr(block_cnt), _stream(stream)))
 
 
+def hsa_select_topp(qpool_blk, cache: DeviceKVCache, t0: int, k_f: int, k_cap: int, p: float, frame_idx,
+                    block_idx, block_cnt, stream=None) -> None:
+    """Selection with the top-p block budget (cap k_cap, threshold p)."""
+    check(lib.cva_hsa_select_topp(_ptr(qpool_blk), ctypes.byref(cache.struct), t0, k_f, k_cap, p,
+                                  _ptr(frame_idx), _ptr(block_idx), _ptr(block_cnt), _stream(stream)))
+
+
 def blocksparse_attn_fwd(q_rot, cache: DeviceKVCache, t0: int, block_idx, block_cnt, k_b_max: int,
                          out, lse=None, workspace=None, stream=None) -> None:
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -351,6 +363,15 @@ def chunk_attention(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0:
     check(lib.cva_chunk_attention(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
                                   ctypes.byref(tables.struct), t0, k_f, k_b, _ptr(workspace),
                                   ws_bytes, _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def chunk_attention_topp(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, k_f: int,
+                         k_cap: int, p: float, workspace, out, lse=None, stream=None) -> None:
+    """chunk_attention with the top-p block budget of hsa_select_topp."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib.cva_chunk_attention_topp(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
+                                       ctypes.byref(tables.struct), t0, k_f, k_cap, p, _ptr(workspace),
+                                       ws_bytes, _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def chunk_attention_noalloc(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, k_f: int,

@@ -449,9 +449,11 @@ int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk
   return CVA_OK;
 }
 
+// Selection launch; topp > 0 switches the second level to the top-p budget
+// with cap k_b.
 static int select_impl(const float* qpool_blk, const cva_kv_cache* cache, int t0, int k_f, int k_b,
                        int32_t* frame_idx, int32_t* block_idx, int32_t* block_cnt, int k_b_max,
-                       cudaStream_t s) {
+                       float topp, cudaStream_t s) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -476,6 +478,8 @@ static int select_impl(const float* qpool_blk, const cva_kv_cache* cache, int t0
   a.k_b = k_b;
   a.k_f_stride = kfe;
   a.k_b_max = k_b_max;
+  a.topp = topp;
+  a.temp_log2 = (float)(1.4426950408889634 / sqrt((double)d.D));
   if (F == 0) {
     // Nothing to pick: every count is zero.
     if (block_cnt) {
@@ -495,7 +499,22 @@ int cva_hsa_select(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0
   if (rc) return rc;
   if (!qpool_blk || !block_idx || !block_cnt) return fail(CVA_EINVAL, "NULL buffer");
   if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
-  return select_impl(qpool_blk, cache, t0, k_f, k_b, frame_idx, block_idx, block_cnt, k_b,
+  return select_impl(qpool_blk, cache, t0, k_f, k_b, frame_idx, block_idx, block_cnt, k_b, 0.f,
+                     static_cast<cudaStream_t>(stream));
+}
+
+static bool topp_ok(float p) { return p > 0.f && p <= 1.f; }
+
+int cva_hsa_select_topp(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0, int32_t k_f,
+                        int32_t k_cap, float p, int32_t* frame_idx, int32_t* block_idx,
+                        int32_t* block_cnt, cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!qpool_blk || !block_idx || !block_cnt) return fail(CVA_EINVAL, "NULL buffer");
+  if (!topp_ok(p)) return fail(CVA_ERANGE, "p must lie in (0, 1]");
+  if (k_cap < 1) return fail(CVA_ERANGE, "k_cap must be >= 1");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  return select_impl(qpool_blk, cache, t0, k_f, k_cap, frame_idx, block_idx, block_cnt, k_cap, p,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -621,7 +640,7 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   if (rc) return rc;
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   if (sparse) {
-    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, s);
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, 0.f, s);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
@@ -697,10 +716,14 @@ int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, 
   return CVA_OK;
 }
 
-int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
-                        const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
-                        void* workspace, size_t ws_bytes, void* out, float* lse,
-                        cva_stream_t stream) {
+}  // extern "C"
+
+// Steps 1-5 from q, k, v; topp > 0 selects blocks by the top-p budget with
+// cap k_b.
+static int chunk_attention_impl(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                                const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                                float topp, void* workspace, size_t ws_bytes, void* out, float* lse,
+                                cva_stream_t stream) {
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!q || !k || !v || !out || !workspace) return fail(CVA_EINVAL, "NULL buffer");
@@ -759,7 +782,7 @@ int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_k
   // step 4
   const bool sparse = !dense && F > 0;
   if (sparse) {
-    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, s);
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, topp, s);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
@@ -769,6 +792,26 @@ int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_k
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;
+}
+
+extern "C" {
+
+int cva_chunk_attention(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                        const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                        void* workspace, size_t ws_bytes, void* out, float* lse,
+                        cva_stream_t stream) {
+  return chunk_attention_impl(q, k, v, cache, tables, t0, k_f, k_b, 0.f, workspace, ws_bytes, out, lse,
+                              stream);
+}
+
+int cva_chunk_attention_topp(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                             const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_cap,
+                             float p, void* workspace, size_t ws_bytes, void* out, float* lse,
+                             cva_stream_t stream) {
+  if (!topp_ok(p)) return fail(CVA_ERANGE, "p must lie in (0, 1]");
+  if (k_f < 1 || k_cap < 1) return fail(CVA_ERANGE, "k_f and k_cap must be >= 1");
+  return chunk_attention_impl(q, k, v, cache, tables, t0, k_f, k_cap, p, workspace, ws_bytes, out, lse,
+                              stream);
 }
 
 }  // extern "C"

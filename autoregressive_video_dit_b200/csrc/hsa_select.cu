@@ -15,6 +15,13 @@
 // the keys in shared memory); it is picked when its rank is below k. The
 // picked positions are written in ascending order by a CTA-wide ordered
 // compaction (warp ballots plus a scan of the per-warp counts).
+//
+// Top-p mode of the second level ("Sparse VideoGen2", section B, centroid
+// top-p, read for key blocks): each candidate's mass is its token count times
+// exp((s - s_max) / sqrt(D)); the count pass also sums the masses of the keys
+// above the candidate, and the candidate is taken when that sum is below p
+// times the total (the top one always, at most k_b). Masses are nonnegative
+// and rounding is monotonic, so the taken set is a prefix of the ranking.
 #include "kernels.cuh"
 
 namespace cva {
@@ -81,6 +88,42 @@ __device__ __forceinline__ int rank_of(const uint64_t* key, int n, int i) {
   return r;
 }
 
+// rank_of plus the fp32 sum of the masses m[] of the keys above key[i]
+// (m[] padded like key[]).
+__device__ __forceinline__ int rank_mass_of(const uint64_t* key, const float* m, int n, int i,
+                                            float* above) {
+  const uint64_t x = key[i];
+  const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(key);
+  const float2* m2 = reinterpret_cast<const float2*>(m);
+  int r = 0;
+  float s = 0.f;
+  for (int j = 0; j < (n + 1) >> 1; ++j) {
+    const ulonglong2 y = k2[j];
+    const float2 w = m2[j];
+    if (y.x > x) { ++r; s += w.x; }
+    if (y.y > x) { ++r; s += w.y; }
+  }
+  *above = s;
+  return r;
+}
+
+// CTA-wide max (is_max) or sum of one float per thread; all threads call it.
+__device__ float cta_reduce(float v, bool is_max, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float y = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = is_max ? fmaxf(v, y) : v + y;
+  }
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kSelWarps; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();
+  return r;
+}
+
 // Ordered compaction over positions 0..n-1: `emit(slot, pos)` for every pos
 // with take(pos), slots counted in ascending pos. Returns the number taken.
 // All threads of the CTA call it.
@@ -119,10 +162,13 @@ __global__ void __launch_bounds__(kSelThreads) hsa_select_kernel(SelectArgs a, i
   const int u = blockIdx.x;
   const int bh = u / d.NQB;
 
-  // smem: keys[nmax + 1] u64, chosen frames [256] i32, row offsets [nmax] i32
+  __shared__ float red[kSelWarps];
+  // smem: keys[nmax + 1] u64, chosen frames [256] i32, row offsets [nmax] i32,
+  // then (top-p) masses [nmax + 1] f32
   uint64_t* key = reinterpret_cast<uint64_t*>(sel_smem);
   int* chosen = reinterpret_cast<int*>(sel_smem + (size_t)(nmax + 1) * 8);
   int* rowoff = chosen + kSelMaxFrames;
+  float* mass = reinterpret_cast<float*>(rowoff + nmax + (nmax & 1));  // 8-byte aligned
 
   float q[D / 32];
   {
@@ -163,26 +209,61 @@ __global__ void __launch_bounds__(kSelThreads) hsa_select_kernel(SelectArgs a, i
   }
   if (tid == 0) key[C] = 0ull;
   __syncthreads();
+  const bool topp = a.topp > 0.f;
+  float smax = -INFINITY;
   for (int b0 = 32 * warp; b0 < C; b0 += 32 * kSelWarps) {
     const float s = score_group<D>(q, b0, C, kblk, rowoff);
     const int c = b0 + lane;
-    if (c < C) key[c] = rank_key(s, c);
+    if (c < C) {
+      key[c] = rank_key(s, c);
+      if (topp) {
+        mass[c] = s;
+        smax = fmaxf(smax, s);
+      }
+    }
+  }
+  float thresh = 0.f;
+  if (topp) {
+    // masses n_c * exp((s_c - s_max) / sqrt(D)); n_c is the block's valid tokens
+    smax = cta_reduce(smax, true, red);  // also orders the mass[] stores
+    const float tail = (float)d.tail;
+    float part = 0.f;
+    for (int c = tid; c < C; c += kSelThreads) {
+      const float n = (c % d.nb == d.nb - 1) ? tail : (float)d.blk;
+      const float m = n * exp2f((mass[c] - smax) * a.temp_log2);
+      mass[c] = m;
+      part += m;
+    }
+    if (tid == 0) mass[C] = 0.f;
+    thresh = a.topp * cta_reduce(part, false, red);
   }
   __syncthreads();
   int32_t* out = a.block_idx + (size_t)u * a.k_b_max;
-  const int nout = compact(
-      C, warp_cnt, [&](int c) { return C <= kb || rank_of(key, C, c) < kb; },
-      [&](int slot, int c) {
-        const int fi = c / d.nb;
-        out[slot] = (a.t_lo + chosen[fi]) * d.nb + (c - fi * d.nb);
-      });
+  auto emit = [&](int slot, int c) {
+    const int fi = c / d.nb;
+    out[slot] = (a.t_lo + chosen[fi]) * d.nb + (c - fi * d.nb);
+  };
+  int nout;
+  if (topp) {
+    nout = compact(
+        C, warp_cnt,
+        [&](int c) {
+          float above;
+          const int r = rank_mass_of(key, mass, C, c, &above);
+          return r < kb && (r == 0 || above < thresh);
+        },
+        emit);
+  } else {
+    nout = compact(C, warp_cnt, [&](int c) { return C <= kb || rank_of(key, C, c) < kb; }, emit);
+  }
   if (tid == 0 && a.block_cnt) a.block_cnt[u] = nout;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   const int kfe = a.k_f < a.F ? a.k_f : a.F;
   const int nmax = a.F > kfe * a.d.nb ? a.F : kfe * a.d.nb;
-  const size_t smem = (size_t)(nmax + 1) * 8 + kSelMaxFrames * 4 + (size_t)nmax * 4;
+  const size_t smem = (size_t)(nmax + 1) * 8 + kSelMaxFrames * 4 + (size_t)nmax * 4 +
+                      (a.topp > 0.f ? (size_t)(nmax + 2) * 4 : 0);
   const int units = a.d.B * a.d.H * a.d.NQB;
   dim3 grid(units);
   cudaError_t e;

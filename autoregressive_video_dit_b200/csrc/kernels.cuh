@@ -51,6 +51,12 @@ struct SelectArgs {
   Dims d;
   int W, t_lo, F;          // history frames t_lo .. t_lo+F-1
   int k_f, k_b, k_f_stride, k_b_max;
+  // Top-p budget of the second level (0: top-k with k = k_b). With p > 0,
+  // k_b is the cap and the blocks are taken in rank order while the softmax
+  // mass (temperature sqrt(D), weighted by token counts) ranked above them
+  // is below p times the total.
+  float topp;
+  float temp_log2;         // log2(e) / sqrt(D)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 

@@ -211,6 +211,23 @@ int cva_hsa_select(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0
                    int32_t k_f, int32_t k_b, int32_t* frame_idx, int32_t* block_idx,
                    int32_t* block_cnt, cva_stream_t stream);
 
+/* Top-p budget for the second level ("Sparse VideoGen2", section B: clusters
+ * sorted by estimated attention and taken until the cumulative share reaches
+ * p). Frames as cva_hsa_select; the candidate blocks of the picked frames
+ * are ranked by q.kb (ties to the lower (t, j)); block c's estimated share is
+ * its valid token count n_c (blk, or the frame's tail for its last block)
+ * times exp((s_c - s_max) / sqrt(D)), over the sum of them all (fp32,
+ * exp2f). In rank order a block is taken while the share ranked above it is
+ * below p: the top block always, at most k_cap blocks.
+ *   block_idx: int32 [B][H][NQB][k_cap], the first block_cnt entries valid
+ *              (ascending ids t*nb + j); the rest are not written.
+ *   block_cnt: int32 [B][H][NQB], 1 .. k_cap (0 without history).
+ * CVA_ERANGE if p is outside (0, 1], k_cap < 1 or k_cap > k_f_eff * nb.
+ * cva_blocksparse_attn_fwd takes these lists with k_b_max = k_cap. */
+int cva_hsa_select_topp(const float* qpool_blk, const cva_kv_cache* cache, int32_t t0,
+                        int32_t k_f, int32_t k_cap, float p, int32_t* frame_idx,
+                        int32_t* block_idx, int32_t* block_cnt, cva_stream_t stream);
+
 /* ---- 5. block-sparse flash attention ("Light Forcing" 2.2, execution) ---- */
 
 /* For query i of query block qb: key set S = valid tokens of the history
@@ -268,6 +285,14 @@ int cva_chunk_attention(const void* q, const void* k, const void* v,
                         const cva_kv_cache* cache, const cva_rope_tables* tables,
                         int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
                         size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
+
+/* cva_chunk_attention with the top-p block budget of cva_hsa_select_topp
+ * (k_f >= 1, cap k_cap, threshold p in (0, 1]); workspace:
+ * cva_chunk_workspace_bytes(shape, k_f, k_cap) bytes. */
+int cva_chunk_attention_topp(const void* q, const void* k, const void* v,
+                             const cva_kv_cache* cache, const cva_rope_tables* tables,
+                             int32_t t0, int32_t k_f, int32_t k_cap, float p, void* workspace,
+                             size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
 /* Steps 1-5 for one chunk starting from the hidden states: the fused QKV
  * projection with Causal-RoPE, append and pooling (cva_qkv_rope_append, the

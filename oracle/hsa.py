@@ -110,6 +110,30 @@ def block_select(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.ndarray
     return cand_ids[pos], gap
 
 
+def topp_ranking(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.ndarray,
+                 nb: int, T_f: int, blk: int):
+    """Candidate blocks of the picked frames in rank order, for the top-p budget.
+
+    Returns ``(ids, scores, above)`` in rank order (score descending, ties to
+    the lower position): the ids ``t * nb + j``, the pooled scores and the
+    share of the estimated attention ranked above each candidate (see
+    :func:`block_select_topp`).
+    """
+    frames_t = np.asarray(frames_t)
+    qbar = np.asarray(qbar, dtype=np.float64)
+    D = qbar.shape[0]
+    s = kbar_blocks.reshape(-1, kbar_blocks.shape[-1]) @ qbar
+    C = s.shape[0]
+    cand_ids = (frames_t[:, None] * nb + np.arange(nb)[None, :]).reshape(-1)
+    tail = T_f - (nb - 1) * blk
+    n = np.tile(np.array([blk] * (nb - 1) + [tail], dtype=np.float64), frames_t.shape[0])
+    order = np.lexsort((np.arange(C), -s))
+    m = n * np.exp((s - s.max()) / math.sqrt(D))
+    ms = m[order]
+    above = (np.cumsum(ms) - ms) / m.sum()
+    return cand_ids[order], s[order], above
+
+
 def block_select_topp(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.ndarray,
                       nb: int, T_f: int, blk: int, p: float, k_cap: int):
     """Second level with a top-p budget instead of a fixed ``k_b``.
@@ -133,28 +157,16 @@ def block_select_topp(qbar: np.ndarray, kbar_blocks: np.ndarray, frames_t: np.nd
     threshold from the cumulative masses around the cut (``inf`` when no
     candidate was left out).
     """
-    frames_t = np.asarray(frames_t)
-    qbar = np.asarray(qbar, dtype=np.float64)
-    D = qbar.shape[0]
-    s = kbar_blocks.reshape(-1, kbar_blocks.shape[-1]) @ qbar
-    C = s.shape[0]
-    cand_ids = (frames_t[:, None] * nb + np.arange(nb)[None, :]).reshape(-1)
-    tail = T_f - (nb - 1) * blk
-    n = np.tile(np.array([blk] * (nb - 1) + [tail], dtype=np.float64), frames_t.shape[0])
-    order = np.lexsort((np.arange(C), -s))
-    m = n * np.exp((s - s.max()) / math.sqrt(D))
-    total = m.sum()
-    ms = m[order]
-    before = np.cumsum(ms) - ms                            # mass ranked above each candidate
-    take = (before < p * total) & (np.arange(C) < k_cap)
+    ids, s, above = topp_ranking(qbar, kbar_blocks, frames_t, nb, T_f, blk)
+    C = ids.shape[0]
+    take = (above < p) & (np.arange(C) < k_cap)
     take[0] = k_cap > 0                                    # at least one block
     r = int(take.sum())
     gap = math.inf
     if r < C:
-        gap = min(rel_gap(s[order[r - 1]], s[order[r]]) if r > 0 else math.inf,
-                  abs(before[r] - p * total) / total,
-                  abs(before[r - 1] - p * total) / total if r > 0 else math.inf)
-    return np.sort(cand_ids[order[:r]]), gap
+        gap = min(rel_gap(s[r - 1], s[r]) if r > 0 else math.inf,
+                  abs(above[r] - p), abs(above[r - 1] - p) if r > 0 else math.inf)
+    return np.sort(ids[:r]), gap
 
 
 # --- chunk budget -----------------------------------------------------------------

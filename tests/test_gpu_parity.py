@@ -46,9 +46,10 @@ def _sub(wl, heads):
     return wl if heads is None else wl.replace(H=len(heads))
 
 
-def _oracle_run(wl, chunk, heads=None, t_begin=0):
+def _oracle_run(wl, chunk, heads=None, t_begin=0, topp=None, cap=None):
     """Oracle over the window's chunks; returns per-chunk bf16 values and the
-    final chunk's path outputs (selection, pooled queries) without attention."""
+    final chunk's path outputs (selection, pooled queries) without attention.
+    With ``topp`` the blocks follow the top-p budget with cap ``cap``."""
     H = wl.H if heads is None else len(heads)
     cache = o_path.FrameCache(wl.B, H, wl.D, wl.T_f, wl.blk, wl.window)
     cache.t_begin = t_begin
@@ -67,8 +68,10 @@ def _oracle_run(wl, chunk, heads=None, t_begin=0):
     x = inputs(wl, chunk, 0, heads, centres)
     q, k, v = (bits_to_f64(x[n]) for n in ("q", "k", "v"))
     k_f, k_b = oracle_budget(wl, chunk, t_begin)
+    if topp is not None:
+        k_b = cap
     out = o_path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0_cur, k_f=k_f, k_b=k_b,
-                           dense=wl.dense, store="bf16", attend_too=False)
+                           dense=wl.dense, store="bf16", attend_too=False, topp=topp)
     out.update(cache=cache, hist=hist, x=x, t0=t0_cur, k_f=k_f, k_b=k_b)
     return out
 
@@ -460,6 +463,165 @@ def test_c5_streaming_window_sampled(ops):
     ok = _selection_ok_mask(run, gb)
     assert ok.mean() >= 0.98, ok.mean()
     rows = sample_rows(wl, 1, np.random.default_rng(6), blocks=range(0, wl.NQB, 4))
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+# ---- top-p block budget ("Sparse VideoGen2", section B) --------------------------------------
+
+def _topp_cap(wl, chunk, which, t_begin=0):
+    """Cap of the top-p lists: every candidate block, or the chunk's top-k budget."""
+    k_f, k_b = lib_budget(wl, chunk, t_begin)
+    kfe = min(k_f, hist_count(wl, chunk, t_begin))
+    return k_f, (kfe * wl.nb if which == "all" else k_b)
+
+
+def _topp_compare(wl, run, gpu_blocks, gpu_cnt, p, cap, tol=1e-4):
+    """Per (b, h, query block): identical to the oracle, or, where it differs,
+    still a valid top-p choice under the oracle's own ranking (a prefix of it
+    whose cut lies within `tol` of p in share, or at a score near-tie).
+    Returns (units, mismatches that are not valid, valid mismatches)."""
+    B, H, NQB, _ = run["blocks"].shape
+    bad = near = 0
+    for b in range(B):
+        for h in range(H):
+            for qb in range(NQB):
+                want = run["blocks"][b, h, qb]
+                want = want[want >= 0]
+                r = int(gpu_cnt[b, h, qb])
+                got = gpu_blocks[b, h, qb, :max(r, 0)]
+                if r == len(want) and np.array_equal(got, want):
+                    continue
+                if run["gap_f"][b, h, qb] < 1e-5:         # the frames themselves were a near tie
+                    near += 1
+                    continue
+                ft = run["frames"][b, h, qb]
+                kb = np.stack([run["cache"].frames[t]["kb"][b, h] for t in ft])
+                ids, sc, above = o_hsa.topp_ranking(run["qbar_blk"][b, h, qb], kb, ft, wl.nb, wl.T_f, wl.blk)
+                lim = min(cap, len(ids))
+                ok = 1 <= r <= lim
+                if ok and not np.array_equal(np.sort(ids[:r]), got):
+                    ok = r < len(ids) and o_hsa.rel_gap(sc[r - 1], sc[r]) < 1e-5
+                if ok and r > 1 and above[r - 1] >= p + tol:
+                    ok = False                               # took a block it should not have
+                if ok and r < lim and above[r] < p - tol:
+                    ok = False                               # stopped before reaching p
+                if ok:
+                    near += 1
+                else:
+                    bad += 1
+    return B * H * NQB, bad, near
+
+
+def _staged_select_topp(ops, wl, run, p, cap):
+    import torch
+    cache = _gpu_cache_from_oracle(ops, wl, run)
+    qd = to_dev(f64_to_bits(_head_major(wl, run["q_rot"])))
+    pb = torch.empty((wl.B, wl.H, wl.NQB, wl.D), dtype=torch.float32, device="cuda")
+    ops.hsa_compress(qd, shape_of(wl), pb)
+    kfe = run["frames"].shape[-1]
+    fi = torch.full((wl.B, wl.H, wl.NQB, max(kfe, 1)), -7, dtype=torch.int32, device="cuda")
+    bi = torch.full((wl.B, wl.H, wl.NQB, cap), -7, dtype=torch.int32, device="cuda")
+    bc = torch.full((wl.B, wl.H, wl.NQB), -7, dtype=torch.int32, device="cuda")
+    ops.hsa_select_topp(pb, cache, run["t0"], run["k_f"], cap, p, fi, bi, bc)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    return fi.cpu().numpy(), bi.cpu().numpy(), bc.cpu().numpy()
+
+
+@pytest.mark.parametrize("p", [0.5, 0.9])
+@pytest.mark.parametrize("key", SMALL_SPARSE)
+def test_hsa_select_topp_staged(ops, key, p):
+    wl = WORKLOADS[key]
+    _, cap = _topp_cap(wl, wl.chunk, "all")
+    run = _oracle_run(wl, wl.chunk, topp=p, cap=cap)
+    fi, bi, bc = _staged_select_topp(ops, wl, run, p, cap)
+    assert np.all((bc >= 1) & (bc <= cap))
+    n, bad, near = _topp_compare(wl, run, bi, bc, p, cap)
+    assert bad == 0 and near <= 0.05 * n, (bad, near, n)
+    kfe = run["frames"].shape[-1]
+    ok = run["gap_f"] >= 1e-5
+    np.testing.assert_array_equal(fi[..., :kfe][ok], run["frames"][ok])
+
+
+def test_hsa_select_topp_cap_binds(ops):
+    # p close to 1 with the cap at the top-k budget: every list is the top-k
+    wl = WORKLOADS["r128"]
+    _, cap = _topp_cap(wl, wl.chunk, "budget")
+    run = _oracle_run(wl, wl.chunk, topp=0.999, cap=cap)
+    _, bi, bc = _staged_select_topp(ops, wl, run, 0.999, cap)
+    n, bad, near = _topp_compare(wl, run, bi, bc, 0.999, cap)
+    assert bad == 0 and near <= 0.05 * n, (bad, near, n)
+    runk = _oracle_run(wl, wl.chunk)
+    full = np.all(run["blocks"] >= 0, axis=-1)
+    assert full.mean() > 0.9
+    np.testing.assert_array_equal(run["blocks"][full], runk["blocks"][full])
+
+
+@pytest.mark.parametrize("chunk,p", [(4, 0.9), (7, 0.7)])
+def test_hsa_select_topp_c3_full_size(ops, chunk, p):
+    wl = WORKLOADS["c3"].with_chunk(chunk)
+    heads = [0, 5, 11]
+    _, cap = _topp_cap(wl, chunk, "all")
+    run = _oracle_run(wl, chunk, heads, topp=p, cap=cap)
+    fi, bi, bc = _staged_select_topp(ops, _sub(wl, heads), run, p, cap)
+    n, bad, near = _topp_compare(_sub(wl, heads), run, bi, bc, p, cap)
+    assert bad == 0 and near <= 0.05 * n, (bad, near, n)
+
+
+def _gpu_stream_topp(ops, wl, upto, p, which):
+    """Fused top-p chunk calls for chunks 2..upto (chunk 1 dense); returns the
+    last chunk's output, its block lists and counts."""
+    import torch
+    shp = shape_of(wl)
+    tabs = _tables(ops, wl)
+    cache = ops.DeviceKVCache(shp, wl.window, 0)
+    centres = key_centres(wl, 0) if wl.keys == "clustered" else None
+    for c in range(1, upto + 1):
+        x = inputs(wl, c, 0, None, centres)
+        out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+        args = [to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]), cache, tabs, wl.t0_of(c)]
+        if c == 1:
+            ws = torch.empty(ops.chunk_workspace_bytes(shp, -1, 0), dtype=torch.uint8, device="cuda")
+            ops.chunk_attention(*args, -1, 0, ws, out)
+            continue
+        k_f, cap = _topp_cap(wl, c, which)
+        ws = torch.empty(ops.chunk_workspace_bytes(shp, k_f, cap), dtype=torch.uint8, device="cuda")
+        ops.chunk_attention_topp(*args, k_f, cap, p, ws, out)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    gb = _ws_blocks(ops, wl, ws, k_f, cap)
+    bhq = wl.B * wl.H * wl.NQB
+    r256 = lambda n: (n + 255) // 256 * 256
+    off = (r256(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r256(bhq * wl.D * 4) + r256(bhq * k_f * 4)
+           + r256(bhq * cap * 4))
+    gc = ws[off:off + bhq * 4].cpu().numpy().view(np.int32).reshape(wl.B, wl.H, wl.NQB)
+    return from_dev(out), gb, gc, cap
+
+
+@pytest.mark.parametrize("key,p", [("c1s", 0.6), ("r64", 0.8), ("r128", 0.5), ("r64s", 0.9)])
+def test_chunk_attention_topp_end_to_end(ops, key, p):
+    wl = WORKLOADS[key]
+    out, gb, gc, cap = _gpu_stream_topp(ops, wl, wl.chunk, p, "all")
+    run = _oracle_run(wl, wl.chunk, topp=p, cap=cap)
+    n, bad, near = _topp_compare(wl, run, gb, gc, p, cap)
+    assert bad == 0 and near <= 0.05 * n, (bad, near, n)
+    ok = np.all(np.where(np.arange(cap) < gc[..., None], gb, -1) == run["blocks"], axis=-1)
+    mx, mean, rel = _e2e_compare(wl, run, out, ok)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
+
+
+def test_c3_topp_end_to_end_sampled(ops):
+    wl = WORKLOADS["c3"].with_chunk(7)
+    p = 0.9
+    out, gb, gc, cap = _gpu_stream_topp(ops, wl, 7, p, "all")
+    heads = [1, 6]
+    run = _oracle_run(wl, 7, heads, topp=p, cap=cap)
+    gb, gc = gb[:, heads], gc[:, heads]
+    n, bad, near = _topp_compare(_sub(wl, heads), run, gb, gc, p, cap)
+    assert bad == 0 and near <= 0.05 * n, (bad, near, n)
+    ok = np.all(np.where(np.arange(cap) < gc[..., None], gb, -1) == run["blocks"], axis=-1)
+    rows = sample_rows(wl, 1, np.random.default_rng(7))
     mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 

@@ -150,6 +150,25 @@ def test_select_rejects_budget_beyond_candidates(ops):
     assert rc == ops.CVA_EINVAL
 
 
+def test_select_topp_rejects_bad_threshold_and_cap(ops):
+    wl = WORKLOADS["r64"]
+    s = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
+    c, _ = _fake_cache(ops, s, wl.window)
+    fake = ctypes.c_void_p(1 << 41)
+    f = ops.lib.cva_hsa_select_topp
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert f(fake, ctypes.byref(c), 6, 4, 8, p, None, fake, fake, None) == ops.CVA_ERANGE
+        assert "p must" in ops.last_error()
+    assert f(fake, ctypes.byref(c), 6, 4, 0, 0.5, None, fake, fake, None) == ops.CVA_ERANGE
+    assert f(fake, ctypes.byref(c), 6, 4, 9, 0.5, None, fake, fake, None) == ops.CVA_ERANGE   # 9 > 8 candidates
+    assert f(None, ctypes.byref(c), 6, 4, 8, 0.5, None, fake, fake, None) == ops.CVA_EINVAL
+    g = ops.lib.cva_chunk_attention_topp
+    assert g(fake, fake, fake, ctypes.byref(c), None, 6, 4, 8, 0.0, fake, 1 << 30, fake, None,
+             None) == ops.CVA_ERANGE
+    assert g(fake, fake, fake, ctypes.byref(c), None, 6, 0, 8, 0.5, fake, 1 << 30, fake, None,
+             None) == ops.CVA_ERANGE
+
+
 def test_attention_rejects_oversized_key_lists(ops):
     # 256 history frames x 25 blocks exceed the per-tile key-unit list
     s = ops.make_shape(1, 1, 128, 30, 52, 3, 64)
