@@ -626,6 +626,38 @@ def test_c3_topp_end_to_end_sampled(ops):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
+# ---- denoising steps of a chunk -----------------------------------------------------------
+
+def test_denoising_passes_leave_no_trace(ops):
+    # chunk 3 runs two noisy passes (other inputs) before its clean pass;
+    # every output from the clean pass on is bit-identical to a stream without them
+    import torch
+    wl = WORKLOADS["r64s"].with_chunk(5)
+    shp = shape_of(wl)
+    tabs = _tables(ops, wl)
+
+    def run(noisy):
+        cache = ops.DeviceKVCache(shp, wl.window, 0)
+        outs = {}
+        for c in range(1, 6):
+            k_f, k_b = lib_budget(wl, c)
+            ws = torch.empty(ops.chunk_workspace_bytes(shp, k_f, k_b), dtype=torch.uint8, device="cuda")
+            layers = [11 + i for i in range(noisy if c == 3 else 0)] + [0]
+            for layer in layers:
+                x = inputs(wl, c, layer)
+                out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+                ops.chunk_attention(to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]), cache, tabs, wl.t0_of(c),
+                                    k_f, k_b, ws, out)
+            outs[c] = from_dev(out)
+        torch.cuda.synchronize()
+        assert ops.device_status() == 0
+        return outs
+
+    a, b = run(0), run(2)
+    for c in (3, 4, 5):
+        np.testing.assert_array_equal(a[c], b[c])
+
+
 # ---- edge cases and errors ------------------------------------------------------------------
 
 def test_zero_blocks_attends_current_chunk_only(ops):

@@ -552,3 +552,28 @@ def test_topp_path_rows_are_top_k_of_their_own_count():
                 kb = np.stack([cache.frames[t]["kb"][b, h] for t in ft])
                 want, _ = hsa.block_select(out["qbar_blk"][b, h, qb], kb, ft, wl.nb, r)
                 np.testing.assert_array_equal(row[:r], want)
+
+
+def test_denoising_passes_leave_no_trace():
+    # every pass of a chunk writes that chunk's frames; only the last (clean)
+    # pass is seen by later chunks, and a pass evicts nothing inside the
+    # chunk's own history
+    wl = WORKLOADS["r64s"].with_chunk(4)
+    def run(noisy_passes):
+        cache = path.FrameCache(wl.B, wl.H, wl.D, wl.T_f, wl.blk, wl.window)
+        outs = {}
+        for c in range(1, 5):
+            t0 = wl.t0_of(c)
+            hist_frames = min(t0, wl.window - wl.Fc)
+            k_f, k_b = hsa.budget(c, hist_frames, wl.nb, dense=False, k_f_max=wl.k_f_max,
+                                  d_base=wl.d_base, d_slope=wl.d_slope, d_pivot=wl.d_pivot)
+            passes = [chunk_inputs(wl, c, layer=7 + i) for i in range(noisy_passes if c == 2 else 0)]
+            passes.append(chunk_inputs(wl, c))
+            for x in passes:
+                q, k, v = (bf16_bits_to_f32(x[n]).astype(np.float64) for n in ("q", "k", "v"))
+                outs[c] = path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0,
+                                         k_f=k_f, k_b=k_b, dense=False)
+        return outs
+    a, b = run(0), run(2)
+    for c in (2, 3, 4):
+        np.testing.assert_array_equal(a[c]["o"], b[c]["o"])
