@@ -46,7 +46,7 @@ class RopeTables(ctypes.Structure):
     _fields_ = [("cos_t", c_void_p), ("sin_t", c_void_p), ("cos_h", c_void_p),
                 ("sin_h", c_void_p), ("cos_w", c_void_p), ("sin_w", c_void_p),
                 ("max_t", c_int32), ("frame_h", c_int32), ("frame_w", c_int32),
-                ("head_dim", c_int32)]
+                ("head_dim", c_int32), ("cs_tok", c_void_p)]
 
 
 class KVCache(ctypes.Structure):
@@ -68,6 +68,7 @@ _SIGS = {
     "cva_device_status": (c_int32, [P(c_int32), c_int32]),
     "cva_rope_axis_pairs": (c_int32, [c_int32, P(c_int32), P(c_int32), P(c_int32)]),
     "cva_rope3d_precompute": (c_int32, [P(RopeCfg)] + [c_void_p] * 6),
+    "cva_rope3d_precompute_tokens": (c_int32, [P(RopeCfg), c_void_p]),
     "cva_rope3d_apply": (c_int32, [c_void_p, c_void_p, P(RopeTables), P(Shape), c_int32, c_int32, c_void_p]),
     "cva_kv_append": (c_int32, [c_void_p, c_void_p, P(KVCache), P(RopeTables), c_int32, c_void_p]),
     "cva_history_frames": (c_int32, [P(KVCache), c_int32, P(c_int32), P(c_int32)]),
@@ -174,6 +175,8 @@ def rope3d_precompute(head_dim: int, max_t: int, frame_h: int, frame_w: int,
     check(lib.cva_rope3d_precompute(ctypes.byref(cfg), *[out[k].ctypes.data for k in
                                                           ("cos_t", "sin_t", "cos_h", "sin_h",
                                                            "cos_w", "sin_w")]))
+    out["cs_tok"] = np.zeros((frame_h, frame_w, head_dim // 2, 2), np.float32)
+    check(lib.cva_rope3d_precompute_tokens(ctypes.byref(cfg), out["cs_tok"].ctypes.data))
     return out
 
 
@@ -240,7 +243,7 @@ class DeviceRopeTables:
         t = self.tensors
         self.struct = RopeTables(_ptr(t["cos_t"]), _ptr(t["sin_t"]), _ptr(t["cos_h"]),
                                  _ptr(t["sin_h"]), _ptr(t["cos_w"]), _ptr(t["sin_w"]),
-                                 max_t, frame_h, frame_w, head_dim)
+                                 max_t, frame_h, frame_w, head_dim, _ptr(t["cs_tok"]))
 
 
 class DeviceKVCache:

@@ -104,6 +104,7 @@ int check_tables(const cva_rope_tables* t, const Dims& d, int t0) {
     return fail(CVA_ERANGE, "rope tables cover %dx%d positions, frame is %dx%d", t->frame_h, t->frame_w, d.Fh, d.Fw);
   if (t0 < 0 || (int64_t)t0 + d.Fc > t->max_t)
     return fail(CVA_ERANGE, "global time %d..%d outside the temporal table (max_t %d)", t0, t0 + d.Fc - 1, t->max_t);
+  if (t->cs_tok && !aligned(t->cs_tok, 16)) return fail(CVA_EINVAL, "cs_tok must be 16-byte aligned");
   return CVA_OK;
 }
 
@@ -111,7 +112,9 @@ RopeTab make_tab(const cva_rope_tables* t, int D) {
   RopeTab r;
   r.cos_t = t->cos_t; r.sin_t = t->sin_t; r.cos_h = t->cos_h; r.sin_h = t->sin_h;
   r.cos_w = t->cos_w; r.sin_w = t->sin_w;
+  r.cs_tok = t->cs_tok;
   axis_pairs(D, &r.pt, &r.ph, &r.pw);
+  r.tab_w = t->frame_w;
   return r;
 }
 
@@ -252,6 +255,39 @@ int cva_rope3d_precompute(const cva_rope_cfg* cfg, float* cos_t, float* sin_t, f
   return CVA_OK;
 }
 
+int cva_rope3d_precompute_tokens(const cva_rope_cfg* cfg, float* cs_tok) {
+  if (!cfg || !cs_tok) return fail(CVA_EINVAL, "NULL argument");
+  if (cfg->head_dim < 6 || cfg->head_dim % 2) return fail(CVA_EINVAL, "head_dim must be even and >= 6");
+  if (cfg->frame_h < 1 || cfg->frame_w < 1) return fail(CVA_EINVAL, "table rows must be >= 1");
+  if (!(cfg->theta > 1.0)) return fail(CVA_EINVAL, "theta must be > 1");
+  int pt, ph, pw;
+  axis_pairs(cfg->head_dim, &pt, &ph, &pw);
+  const int np = cfg->head_dim / 2;
+  // the same values as the per-axis tables: (float)cos/sin of pos * rate in double
+  for (int h = 0; h < cfg->frame_h; ++h) {
+    for (int w = 0; w < cfg->frame_w; ++w) {
+      float* e = cs_tok + ((size_t)h * cfg->frame_w + w) * np * 2;
+      for (int p = 0; p < np; ++p) {
+        int pos = 0, j = 0, pa = 1;
+        if (p < pt) {
+          e[2 * p] = 1.f;
+          e[2 * p + 1] = 0.f;
+          continue;
+        } else if (p < pt + ph) {
+          pos = h; j = p - pt; pa = ph;
+        } else {
+          pos = w; j = p - pt - ph; pa = pw;
+        }
+        const double rate = pow(cfg->theta, -(2.0 * j) / (2.0 * pa));
+        const double ang = (double)pos * rate;
+        e[2 * p] = (float)cos(ang);
+        e[2 * p + 1] = (float)sin(ang);
+      }
+    }
+  }
+  return CVA_OK;
+}
+
 int cva_history_frames(const cva_kv_cache* cache, int32_t t0, int32_t* t_lo, int32_t* count) {
   int rc = check_cache(cache);
   if (rc) return rc;
@@ -385,9 +421,14 @@ int cva_kv_append(const void* k, const void* v, const cva_kv_cache* cache,
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "kv_append frame pool launch");
 }
 
-int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden, const cva_kv_cache* cache,
-                        const cva_rope_tables* tables, int32_t t0, void* q_rot, float* qpool_blk,
-                        cva_stream_t stream) {
+}  // extern "C"
+
+// The fused projection; with frame_pool the frame means of the new cache
+// frames follow in a second launch (the fused chunk call has the attention
+// launch compute them instead).
+static int qkv_rope_append_impl(const void* x, const void* w_qkv, int32_t hidden, const cva_kv_cache* cache,
+                                const cva_rope_tables* tables, int32_t t0, void* q_rot, float* qpool_blk,
+                                cva_stream_t stream, bool frame_pool) {
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!x || !w_qkv || !q_rot || !tables) return fail(CVA_EINVAL, "x, w_qkv, q_rot or tables is NULL");
@@ -418,9 +459,18 @@ int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden, const 
   cudaError_t e = launch_qkv_rope(a, x, w_qkv, s, &why);
   if (e == cudaErrorInvalidValue && why[0]) return fail(CVA_ELAUNCH, "qkv_rope_append: %s", why);
   if (e != cudaSuccess) return cuda_fail(e, "qkv_rope_append launch");
+  if (!frame_pool) return CVA_OK;
   FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
   e = launch_frame_pool(fp, s);
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "qkv_rope_append frame pool launch");
+}
+
+extern "C" {
+
+int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden, const cva_kv_cache* cache,
+                        const cva_rope_tables* tables, int32_t t0, void* q_rot, float* qpool_blk,
+                        cva_stream_t stream) {
+  return qkv_rope_append_impl(x, w_qkv, hidden, cache, tables, t0, q_rot, qpool_blk, stream, true);
 }
 
 int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk, float* qpool_frm,
@@ -539,9 +589,11 @@ static int sm_count() {
   return counts[dev];
 }
 
+// frame_means: the launch also writes the frame means of the chunk's cache
+// frames (its spare warps), from the block means the chunk's append wrote.
 static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const int32_t* block_idx,
                      const int32_t* block_cnt, int k_b_max, void* out, float* lse, void* split_ws,
-                     size_t split_bytes, cudaStream_t s) {
+                     size_t split_bytes, cudaStream_t s, bool frame_means = false) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -561,6 +613,10 @@ static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const
   a.F = F;
   a.MT = (d.Fc * d.T_pad + 127) / 128;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d.D));
+  if (frame_means) {
+    a.kpool_blk = cache->kpool_blk;
+    a.kpool_frm = cache->kpool_frm;
+  }
   // Tail split: the tiles of the last, partial wave are cut into key-range
   // pieces so that they fill the SMs (needs the scratch; else unsplit).
   const int tiles = a.MT * d.B * d.H;
@@ -636,7 +692,7 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   cudaError_t e = stage_mark(0, s);
   if (e != cudaSuccess) return cuda_fail(e, "stage event");
   // steps 1-3: projection, rotation, append and pooling in the fused kernel
-  rc = cva_qkv_rope_append(x, w_qkv, hidden, cache, tables, t0, q_rot, sparse ? qpool : nullptr, stream);
+  rc = qkv_rope_append_impl(x, w_qkv, hidden, cache, tables, t0, q_rot, sparse ? qpool : nullptr, stream, false);
   if (rc) return rc;
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   if (sparse) {
@@ -645,7 +701,7 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;
@@ -774,9 +830,6 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
   if (e != cudaSuccess) return cuda_fail(e, "stage event");
   e = launch_rope_pool(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "chunk_attention rope/append launch");
-  FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
-  e = launch_frame_pool(fp, s);
-  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention frame pool launch");
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
 
   // step 4
@@ -786,9 +839,9 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
-  // step 5
+  // step 5 (with the frame means of the new cache frames)
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;

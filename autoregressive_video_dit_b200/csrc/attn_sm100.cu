@@ -620,6 +620,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           a.lse[(size_t)bh * d.Lq + n_tok] = (M + log2f(l_tot)) * 0.69314718055994531f;
       }
     }
+  } else if (a.kpool_frm) {
+    // ------------------------------------------------------------ spare warps
+    // Frame means of the chunk's new cache frames from their block means
+    // (written by the previous launch), in the order of frame_pool_kernel:
+    // sum_j count_j * mean_j / T_f. CTA i takes frames i, i + grid, ...
+    const Dims& d = a.d;
+    const int nfr = d.B * d.H * d.Fc;
+    const int c0 = tid - (kMmaWarp + 1) * 32;
+    constexpr int kSpare = kAttnThreads - (kMmaWarp + 1) * 32;
+    for (int fr = blockIdx.x; fr < nfr; fr += gridDim.x) {
+      const int fbh = fr / d.Fc;
+      const int f = fr - fbh * d.Fc;
+      const int fslot = (a.t0 + f) % a.W;
+      const float* src = a.kpool_blk + ((size_t)fbh * a.W + fslot) * d.nb * D;
+      float* dst = a.kpool_frm + ((size_t)fbh * a.W + fslot) * D;
+      for (int c = c0; c < D; c += kSpare) {
+        float sum = 0.f;
+        for (int j = 0; j < d.nb; ++j) {
+          const float cnt = (float)((j == d.nb - 1) ? d.tail : d.blk);
+          sum += cnt * src[(size_t)j * D + c];
+        }
+        dst[c] = sum / (float)d.T_f;
+      }
+    }
   }
 
   tc_fence_before();

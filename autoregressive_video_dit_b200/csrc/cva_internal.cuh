@@ -42,7 +42,9 @@ struct RopeTab {
   const float* cos_t; const float* sin_t;
   const float* cos_h; const float* sin_h;
   const float* cos_w; const float* sin_w;
+  const float* cs_tok;  // (cos, sin) per (h, w, pair) [tab_h][tab_w][D/2][2], or nullptr
   int pt, ph, pw;
+  int tab_w;            // w positions of the tables (row stride of cs_tok in positions)
 };
 
 // Latch the first device-side error of the library.

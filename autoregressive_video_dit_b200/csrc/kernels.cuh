@@ -78,6 +78,10 @@ struct AttnArgs {
   int Qf, pieces;
   float* part_o;             // [piece slot][128][D] fp32, unnormalised
   float* part_ml;            // [piece slot][128][2] running max (log2 units), sum
+  // Optional: frame means of the chunk's cache frames (t0 .. t0+Fc-1) from
+  // their block means, computed by the CTAs' spare warps.
+  const float* kpool_blk;    // [B][H][W][nb][D]
+  float* kpool_frm;          // [B][H][W][D], or nullptr
 };
 // Piece slots of the tail split (one per SM at most).
 constexpr int kAttnMaxPieces = 160;

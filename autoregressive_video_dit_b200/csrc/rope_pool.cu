@@ -8,19 +8,94 @@
 // contiguous tables. "Light Forcing", section 2.2 (token compression):
 // queries and keys are mean-pooled per block and per frame.
 //
-// One CTA handles one (batch*head, frame, block) tile of up to three
-// tensors (Q, K, V) in a single pass over HBM: each thread owns 8
-// consecutive elements (one 16-byte vector) of a row, so a warp reads and
-// writes whole 256-byte rows. Block sums are reduced in a fixed order
-// (deterministic), from the bf16 values actually stored.
+// One CTA handles one (batch*head, frame, block) of up to three tensors
+// (Q, K, V) in a single pass over HBM. Each thread owns 8 consecutive
+// elements (one 16-byte vector) of a row, so a warp reads and writes whole
+// rows; a thread issues the loads of its rows of a batch, for all tensors,
+// together with its 32-byte entries of the per-position (cos, sin) table,
+// before it uses any of them. The job
+// properties (which tensors are rotated or pooled) are template parameters,
+// so the per-row work is the loads, the rotation, the pooling sums and the
+// stores. Block sums are reduced in a fixed order from the bf16 values
+// actually stored (deterministic). Frame means of the block means are a
+// separate step (frame_pool_kernel, or the attention kernel's spare warps
+// in the fused chunk call).
 #include "kernels.cuh"
 
 namespace cva {
 
+// Compile-time job properties: rotation and block pooling of jobs 0 and 1
+// (job 2, when present, is a plain copy).
+enum : int { kRot0 = 1, kRot1 = 2, kPool0 = 4, kPool1 = 8 };
+
+// Addressing of one job in a block: the thread's vector in its first row
+// and the row stride (elements).
+struct JobRows {
+  const uint16_t* src;
+  uint16_t* dst;
+  int sstride, dstride;
+  bool tok_dst;
+};
+
 template <int D>
-__global__ void __launch_bounds__(256) rope_pool_kernel(RopePoolArgs a) {
-  constexpr int kCG = D / 8;          // column groups (16-byte vectors) per row
-  constexpr int kRP = 256 / kCG;      // rows per pass
+__device__ __forceinline__ JobRows job_rows(const StreamJob& job, const Dims& d, int b, int h, int bh,
+                                            int f, int slot, int W, int row, int col) {
+  JobRows r;
+  if (job.src_layout == kTokenMajor) {
+    r.src = job.src + (((size_t)b * d.Lq + (size_t)f * d.T_f + row) * d.H + h) * D + col;
+    r.sstride = d.H * D;
+  } else {
+    r.src = job.src + ((size_t)bh * d.Fc * d.T_pad + (size_t)f * d.T_pad + row) * D + col;
+    r.sstride = D;
+  }
+  r.dst = nullptr;
+  r.dstride = D;
+  r.tok_dst = false;
+  if (job.dst) {
+    if (job.dst_layout == kTokenMajor) {
+      r.dst = job.dst + (((size_t)b * d.Lq + (size_t)f * d.T_f + row) * d.H + h) * D + col;
+      r.dstride = d.H * D;
+      r.tok_dst = true;
+    } else if (job.dst_layout == kHeadMajor) {
+      r.dst = job.dst + ((size_t)bh * d.Fc * d.T_pad + (size_t)f * d.T_pad + row) * D + col;
+    } else {
+      r.dst = job.dst + (((size_t)bh * W + slot) * d.T_pad + row) * D + col;
+    }
+  }
+  return r;
+}
+
+// Rotation of 4 adjacent pairs packed as bf16: (x0, x1) -> (x0 c - x1 s, x0 s + x1 c).
+__device__ __forceinline__ uint4 rotate4(uint4 v, const float (&c)[4], const float (&s)[4]) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x0 = bf16_lo(in[i]);
+    const float x1 = bf16_hi(in[i]);
+    out[i] = pack_bf16(x0 * c[i] - x1 * s[i], x0 * s[i] + x1 * c[i]);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__device__ __forceinline__ void pool_add(float (&acc)[8], uint4 y) {
+  acc[0] += bf16_lo(y.x); acc[1] += bf16_hi(y.x);
+  acc[2] += bf16_lo(y.y); acc[3] += bf16_hi(y.y);
+  acc[4] += bf16_lo(y.z); acc[5] += bf16_hi(y.z);
+  acc[6] += bf16_lo(y.w); acc[7] += bf16_hi(y.w);
+}
+
+// NJ jobs (1..3) with the properties FL; rows of a block in batches of ROWS;
+// at least MINB CTAs per SM.
+template <int D, int NJ, int FL, int ROWS, int MINB>
+__global__ void __launch_bounds__(256, MINB) rope_pool_kernel(RopePoolArgs a) {
+  constexpr int kCG = D / 8;         // column groups (16-byte vectors) per row
+  constexpr int kRP = 256 / kCG;     // rows per pass
+  constexpr int kPass = ROWS / kRP;  // passes per batch
+  constexpr bool kRot[3] = {(FL & kRot0) != 0, (FL & kRot1) != 0, false};
+  constexpr bool kPool[3] = {(FL & kPool0) != 0, (FL & kPool1) != 0, false};
+  constexpr bool kAnyRot = (FL & (kRot0 | kRot1)) != 0;
+  static_assert(NJ >= 1 && NJ <= 3 && kPass >= 1, "bad configuration");
   __shared__ float red[kRP][D];
 
   const Dims& d = a.d;
@@ -30,113 +105,163 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(RopePoolArgs a) {
   const int b = bh / d.H;
   const int h = bh - b * d.H;
   const int tid = threadIdx.x;
-  const int cg = tid % kCG;
+  const int cgi = tid % kCG;
   const int rg = tid / kCG;
   const int valid = (j == d.nb - 1) ? d.tail : d.blk;
   const int t = a.t0 + f;
   const int slot = t % a.W;
+  const int row0 = j * d.blk;
 
-  // Rotary table lookups of this thread's 4 pairs: axis and local index.
-  const float* ctab[4];
-  const float* stab[4];
-  int axis[4];
-  int pstride[4];
+  JobRows jr[NJ];
+#pragma unroll
+  for (int jb = 0; jb < NJ; ++jb) jr[jb] = job_rows<D>(a.job[jb], d, b, h, bh, f, slot, a.W, row0 + rg, cgi * 8);
+
+  // This thread's 4 pairs: axis (0 t, 1 h, 2 w) and table column.
+  int axis[4], col[4];
+  float ct[4], st[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int p = cg * 4 + i;
+    const int p = cgi * 4 + i;
     if (p < a.tab.pt) {
-      axis[i] = 0; ctab[i] = a.tab.cos_t + p; stab[i] = a.tab.sin_t + p; pstride[i] = a.tab.pt;
+      axis[i] = 0; col[i] = p;
     } else if (p < a.tab.pt + a.tab.ph) {
-      const int q = p - a.tab.pt;
-      axis[i] = 1; ctab[i] = a.tab.cos_h + q; stab[i] = a.tab.sin_h + q; pstride[i] = a.tab.ph;
+      axis[i] = 1; col[i] = p - a.tab.pt;
     } else {
-      const int q = p - a.tab.pt - a.tab.ph;
-      axis[i] = 2; ctab[i] = a.tab.cos_w + q; stab[i] = a.tab.sin_w + q; pstride[i] = a.tab.pw;
+      axis[i] = 2; col[i] = p - a.tab.pt - a.tab.ph;
+    }
+  }
+  const float* cs_tok = a.tab.cs_tok;  // per-position table, or nullptr (per-axis lookups)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ct[i] = 1.f;
+    st[i] = 0.f;
+    if (kAnyRot && axis[i] == 0) {
+      ct[i] = __ldg(a.tab.cos_t + (size_t)t * a.tab.pt + col[i]);
+      st[i] = __ldg(a.tab.sin_t + (size_t)t * a.tab.pt + col[i]);
     }
   }
 
-  for (int jb = 0; jb < a.njobs; ++jb) {
-    const StreamJob job = a.job[jb];
-    float acc[8];
+  float acc[2][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int jb = 0; jb < 2; ++jb)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[jb][i] = 0.f;
+  int hh = 0, ww = 0;
+  if (kAnyRot) {
+    hh = (row0 + rg) / d.Fw;
+    ww = row0 + rg - hh * d.Fw;
+  }
 
-    for (int r = rg; r < d.blk; r += kRP) {
-      const int rr = j * d.blk + r;            // row inside the frame (padded)
-      uint4 y = make_uint4(0u, 0u, 0u, 0u);
-      if (r < valid) {
-        size_t src_off;
-        if (job.src_layout == kTokenMajor) {
-          const size_t n = (size_t)f * d.T_f + rr;
-          src_off = (((size_t)b * d.Lq + n) * d.H + h) * D;
-        } else {
-          src_off = ((size_t)bh * d.Fc * d.T_pad + (size_t)f * d.T_pad + rr) * D;
-        }
-        const uint4 x = *reinterpret_cast<const uint4*>(job.src + src_off + cg * 8);
-        if (job.rotate) {
-          const int hh = rr / d.Fw;
-          const int ww = rr - hh * d.Fw;
-          const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
-          uint32_t yout[4];
+  for (int g = 0; g < d.blk; g += ROWS) {
+    uint4 x[NJ][kPass];
+    float4 cs4[kPass][2];  // (c0, s0, c1, s1), (c2, s2, c3, s3) of this thread's pairs
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int pos = axis[i] == 0 ? t : (axis[i] == 1 ? hh : ww);
-            const float c = __ldg(ctab[i] + (size_t)pos * pstride[i]);
-            const float s = __ldg(stab[i] + (size_t)pos * pstride[i]);
-            const float x0 = bf16_lo(xin[i]);
-            const float x1 = bf16_hi(xin[i]);
-            yout[i] = pack_bf16(x0 * c - x1 * s, x0 * s + x1 * c);
-          }
-          y = make_uint4(yout[0], yout[1], yout[2], yout[3]);
-        } else {
-          y = x;
-        }
-        if (job.pool) {
-          acc[0] += bf16_lo(y.x); acc[1] += bf16_hi(y.x);
-          acc[2] += bf16_lo(y.y); acc[3] += bf16_hi(y.y);
-          acc[4] += bf16_lo(y.z); acc[5] += bf16_hi(y.z);
-          acc[6] += bf16_lo(y.w); acc[7] += bf16_hi(y.w);
-        }
+    for (int p = 0; p < kPass; ++p) {
+      cs4[p][0] = make_float4(1.f, 0.f, 1.f, 0.f);
+      cs4[p][1] = make_float4(1.f, 0.f, 1.f, 0.f);
+    }
+    const bool full = g + ROWS <= valid;
+#pragma unroll
+    for (int p = 0; p < kPass; ++p) {
+      const bool live = full || g + p * kRP + rg < valid;
+#pragma unroll
+      for (int jb = 0; jb < NJ; ++jb) {
+        x[jb][p] = make_uint4(0u, 0u, 0u, 0u);
+        if (live) x[jb][p] = __ldcs(reinterpret_cast<const uint4*>(jr[jb].src + (size_t)(g + p * kRP) * jr[jb].sstride));
       }
-      if (job.dst) {
-        if (job.dst_layout == kTokenMajor) {
-          if (r < valid) {
-            const size_t n = (size_t)f * d.T_f + rr;
-            *reinterpret_cast<uint4*>(job.dst + (((size_t)b * d.Lq + n) * d.H + h) * D + cg * 8) = y;
-          }
-        } else if (job.dst_layout == kHeadMajor) {
-          *reinterpret_cast<uint4*>(
-              job.dst + ((size_t)bh * d.Fc * d.T_pad + (size_t)f * d.T_pad + rr) * D + cg * 8) = y;
-        } else {
-          *reinterpret_cast<uint4*>(
-              job.dst + (((size_t)bh * a.W + slot) * d.T_pad + rr) * D + cg * 8) = y;
+    }
+    if (kAnyRot && cs_tok && cgi * 4 + 3 >= a.tab.pt) {  // threads with a spatial pair
+      int h2 = hh, w2 = ww;
+#pragma unroll
+      for (int p = 0; p < kPass; ++p) {
+        const bool live = full || g + p * kRP + rg < valid;
+        if (live) {
+          const float4* e = reinterpret_cast<const float4*>(cs_tok + ((size_t)(h2 * a.tab.tab_w + w2) * (D / 2) + 4 * cgi) * 2);
+          cs4[p][0] = __ldg(e);
+          cs4[p][1] = __ldg(e + 1);
+        }
+        w2 += kRP;
+        while (w2 >= d.Fw) {
+          w2 -= d.Fw;
+          ++h2;
         }
       }
     }
-
-    if (job.pool) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) red[rg][cg * 8 + i] = acc[i];
-      __syncthreads();
-      if (tid < D) {
-        float s = 0.f;
+    for (int p = 0; p < kPass; ++p) {
+      const bool live = full || g + p * kRP + rg < valid;
+      float c[4], s[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        c[i] = kAnyRot ? ct[i] : 1.f;
+        s[i] = kAnyRot ? st[i] : 0.f;
+      }
+      if (kAnyRot && cs_tok) {
+        const float e[8] = {cs4[p][0].x, cs4[p][0].y, cs4[p][0].z, cs4[p][0].w,
+                            cs4[p][1].x, cs4[p][1].y, cs4[p][1].z, cs4[p][1].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (axis[i] != 0) {
+            c[i] = e[2 * i];
+            s[i] = e[2 * i + 1];
+          }
+        }
+      } else if (kAnyRot && live) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (axis[i] == 1) {
+            c[i] = __ldg(a.tab.cos_h + hh * a.tab.ph + col[i]);
+            s[i] = __ldg(a.tab.sin_h + hh * a.tab.ph + col[i]);
+          } else if (axis[i] == 2) {
+            c[i] = __ldg(a.tab.cos_w + ww * a.tab.pw + col[i]);
+            s[i] = __ldg(a.tab.sin_w + ww * a.tab.pw + col[i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int jb = 0; jb < NJ; ++jb) {
+        uint4 y = x[jb][p];
+        if (kRot[jb] && live) y = rotate4(y, c, s);
+        if (kPool[jb]) pool_add(acc[jb], y);
+        if (jr[jb].dst && (live || !jr[jb].tok_dst))
+          *reinterpret_cast<uint4*>(jr[jb].dst + (size_t)(g + p * kRP) * jr[jb].dstride) = y;
+      }
+      if (kAnyRot) {
+        ww += kRP;
+        while (ww >= d.Fw) {
+          ww -= d.Fw;
+          ++hh;
+        }
+      }
+    }
+  }
+
+  // block means, reduced over the pass rows in a fixed order
+#pragma unroll
+  for (int jb = 0; jb < 2; ++jb) {
+    if (!kPool[jb] || jb >= NJ) continue;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[rg][cgi * 8 + i] = acc[jb][i];
+    __syncthreads();
+    if (tid < D) {
+      float sum = 0.f;
 #pragma unroll 4
-        for (int g = 0; g < kRP; ++g) s += red[g][tid];
-        const float mean = s / (float)valid;
-        size_t off;
-        if (job.pool_layout == kPoolChunk) {
-          off = ((size_t)bh * d.NQB + (size_t)f * d.nb + j) * D + tid;
-        } else {
-          off = (((size_t)bh * a.W + slot) * d.nb + j) * D + tid;
-        }
-        job.pool[off] = mean;
+      for (int gg = 0; gg < kRP; ++gg) sum += red[gg][tid];
+      const StreamJob& job = a.job[jb];
+      size_t off;
+      if (job.pool_layout == kPoolChunk) {
+        off = ((size_t)bh * d.NQB + (size_t)f * d.nb + j) * D + tid;
+      } else {
+        off = (((size_t)bh * a.W + slot) * d.nb + j) * D + tid;
       }
-      __syncthreads();
+      job.pool[off] = sum / (float)valid;
     }
+    __syncthreads();
   }
 }
 
-// Frame means from block means: sum_j count_j * mean_j / T_f, in block order.
+// Frame means from block means: sum_j count_j * mean_j / T_f, in block order
+// (for block means written by the fused QKV projection).
 __global__ void frame_pool_kernel(FramePoolArgs a) {
   const Dims& d = a.d;
   const int f = blockIdx.x;
@@ -163,14 +288,41 @@ __global__ void frame_pool_kernel(FramePoolArgs a) {
 
 // ---- host-side launchers (called from api.cu) -----------------------------
 
-cudaError_t launch_rope_pool(const RopePoolArgs& a, cudaStream_t stream) {
+template <int D, int NJ, int FL>
+static cudaError_t launch_rope_pool_t(const RopePoolArgs& a, cudaStream_t stream) {
+  constexpr int kRows = D == 128 ? 16 : 32;  // one pass of 256 threads
   dim3 grid(a.d.Fc * a.d.nb, a.d.B * a.d.H);
-  if (a.d.D == 128) {
-    rope_pool_kernel<128><<<grid, 256, 0, stream>>>(a);
-  } else {
-    rope_pool_kernel<64><<<grid, 256, 0, stream>>>(a);
-  }
+  rope_pool_kernel<D, NJ, FL, kRows, 3><<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_rope_pool_d(const RopePoolArgs& a, int fl, cudaStream_t stream) {
+  switch (a.njobs * 16 + fl) {
+    // chunk call: Q rotated (pooled when sparse), K rotated and pooled, V copied
+    case 3 * 16 + (kRot0 | kRot1 | kPool1): return launch_rope_pool_t<D, 3, kRot0 | kRot1 | kPool1>(a, stream);
+    case 3 * 16 + (kRot0 | kRot1 | kPool0 | kPool1):
+      return launch_rope_pool_t<D, 3, kRot0 | kRot1 | kPool0 | kPool1>(a, stream);
+    // append: K (rotated or not) pooled, V copied
+    case 2 * 16 + (kRot0 | kPool0): return launch_rope_pool_t<D, 2, kRot0 | kPool0>(a, stream);
+    case 2 * 16 + kPool0: return launch_rope_pool_t<D, 2, kPool0>(a, stream);
+    // rotation alone; pooling alone
+    case 1 * 16 + kRot0: return launch_rope_pool_t<D, 1, kRot0>(a, stream);
+    case 1 * 16 + kPool0: return launch_rope_pool_t<D, 1, kPool0>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_rope_pool(const RopePoolArgs& a, cudaStream_t stream) {
+  if (a.njobs < 1 || a.njobs > 3) return cudaErrorInvalidValue;
+  if ((int64_t)a.d.B * a.d.H > 65535) return cudaErrorInvalidConfiguration;
+  if (a.njobs == 3 && (a.job[2].pool || a.job[2].rotate)) return cudaErrorInvalidValue;
+  int fl = 0;
+  for (int jb = 0; jb < a.njobs && jb < 2; ++jb) {
+    if (a.job[jb].rotate) fl |= jb == 0 ? kRot0 : kRot1;
+    if (a.job[jb].pool) fl |= jb == 0 ? kPool0 : kPool1;
+  }
+  return a.d.D == 128 ? launch_rope_pool_d<128>(a, fl, stream) : launch_rope_pool_d<64>(a, fl, stream);
 }
 
 cudaError_t launch_frame_pool(const FramePoolArgs& a, cudaStream_t stream) {

@@ -138,14 +138,17 @@ def attention_flops(st):
     if st["k_f"] < 0 or st["F"] == 0:
         keys = st["F"] * wl.T_f + wl.Lq
         return 4.0 * wl.D * wl.B * wl.H * float(qcount.sum()) * keys
-    blocks = block_lists(st)                                          # [B,H,NQB,k_b]
+    blocks, cnt = block_lists(st)                                     # [B,H,NQB,k_b], [B,H,NQB]
     tail = wl.T_f - (wl.nb - 1) * wl.blk
     valid = np.where(blocks % wl.nb == wl.nb - 1, tail, wl.blk)
+    valid = np.where(np.arange(st["k_b"]) < cnt[..., None], valid, 0)  # top-p lists are shorter
     keys = valid.sum(axis=-1) + wl.Lq                                 # [B,H,NQB]
     return 4.0 * wl.D * float((keys * qcount[None, None, :]).sum())
 
 
 def block_lists(st):
+    """Block lists and their lengths from the chunk workspace (its layout:
+    rotated q, pooled q, frame lists, block lists, block counts)."""
     import numpy as np
     wl = st["wl"]
     bhq = wl.B * wl.H * wl.NQB
@@ -153,7 +156,10 @@ def block_lists(st):
     off = (r(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r(bhq * wl.D * 4)
            + r(bhq * max(st["k_f"], 0) * 4))
     raw = st["ws"][off:off + bhq * st["k_b"] * 4].cpu().numpy().view(np.int32)
-    return raw.reshape(wl.B, wl.H, wl.NQB, st["k_b"]).astype(np.int64)
+    off += r(bhq * st["k_b"] * 4)
+    cnt = st["ws"][off:off + bhq * 4].cpu().numpy().view(np.int32)
+    return (raw.reshape(wl.B, wl.H, wl.NQB, st["k_b"]).astype(np.int64),
+            cnt.reshape(wl.B, wl.H, wl.NQB).astype(np.int64))
 
 
 def attention_launches(wl):
@@ -522,11 +528,11 @@ def run_cuda(args):
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": f"{peak_src} bf16 burst"},
-        "roofline_hbm": {"kernel": "rope_pool_kernel + frame_pool_kernel", "bound": "hbm",
+        "roofline_hbm": {"kernel": "rope_pool_kernel", "bound": "hbm",
                          "achieved": rb / (rope_avg * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": rb / (rope_avg * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
                          "algorithmic_bytes": rb},
-        "gpu_launches": n * (2 + (1 if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
+        "gpu_launches": n * (1 + (1 if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
         "clocks": clocks,
     }
     if e2e:
@@ -554,20 +560,29 @@ def run_sweep(args):
     flush = L2Flush()
     # third schedule: density from the noise level (s_base 0.8, target 0.75)
     noise = ops.cag_noise_densities(base.chunks, base.Fc, base.window, base.nb, 0.8, 0.75)
-    schedules = [("literal", base.d_slope, None), ("mirrored", -base.d_slope, None),
-                 ("noise s_base=0.8 s_target=0.75", base.d_slope, noise)]
-    for sched, slope, dens in schedules:
+    # fourth: the top-p budget (p = 0.9, capped at every candidate block)
+    schedules = [("literal", base.d_slope, None, None), ("mirrored", -base.d_slope, None, None),
+                 ("noise s_base=0.8 s_target=0.75", base.d_slope, noise, None),
+                 ("top-p p=0.9", base.d_slope, None, 0.9)]
+    for sched, slope, dens, topp in schedules:
         for chunk in range(1, base.chunks + 1):
             wl = base.replace(d_slope=slope).with_chunk(chunk)
+            hist = min(base.Fc * (chunk - 1), base.window - base.Fc)
             if dens is not None and chunk >= 2:
-                hist = min(base.Fc * (chunk - 1), base.window - base.Fc)
                 _, kb = ops.cag_density_budget(chunk, hist, base.nb, base.k_f_max, dens[chunk])
                 wl = wl.replace(k_b_fixed=kb)
+            if topp is not None and chunk >= 2:
+                wl = wl.replace(k_b_fixed=min(base.k_f_max, hist) * base.nb)   # the cap
             st = setup_workload(args, layer=0, wl=wl)
+            use_topp = topp is not None and st["F"] > 0
 
             def step():
-                ops.chunk_attention(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0,
-                                    st["k_f"], st["k_b"], st["ws"], st["out"])
+                if use_topp:
+                    ops.chunk_attention_topp(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0,
+                                             st["k_f"], st["k_b"], topp, st["ws"], st["out"])
+                else:
+                    ops.chunk_attention(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0,
+                                        st["k_f"], st["k_b"], st["ws"], st["out"])
 
             for _ in range(max(args.warmup, 1)):
                 flush.zero_()
@@ -575,12 +590,16 @@ def run_sweep(args):
             torch.cuda.synchronize()
             assert ops.device_status() == 0
             flops = attention_flops(st)
+            mean_blocks = st["k_b"]
+            if use_topp:
+                mean_blocks = float(block_lists(st)[1].mean())
             step_ms, rope_ms, sel_ms, attn_ms = time_steps(step, flush, args.steps, stream)
             assert ops.device_status() == 0
             ms = statistics.median(step_ms)
             print(json.dumps({
                 "mode": "schedule sweep", "workload": wl.key, "schedule": sched, "chunk": chunk,
                 "history_frames": st["F"], "k_f": st["k_f"], "k_b": st["k_b"],
+                "mean_blocks": mean_blocks,
                 "ms": ms, "attention_ms": statistics.median(attn_ms),
                 "select_us": 1e3 * statistics.median(sel_ms),
                 "select_share": statistics.median(sel_ms) / ms,

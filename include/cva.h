@@ -99,12 +99,18 @@ typedef struct cva_rope_cfg {
 } cva_rope_cfg;
 
 /* Device copies of the rotary tables (host struct holding device pointers).
- * Each table is fp32 row-major [positions][pairs of that axis]. */
+ * Each table is fp32 row-major [positions][pairs of that axis]. cs_tok is
+ * optional (NULL: not used): the spatial tables expanded per position,
+ * (cos, sin) interleaved, [frame_h][frame_w][head_dim/2][2] floats with
+ * (1, 0) for the temporal pairs (cva_rope3d_precompute_tokens), 16-byte
+ * aligned; with it the rotation reads one contiguous 32-byte entry per 4
+ * pairs instead of looking each pair up. Results are identical. */
 typedef struct cva_rope_tables {
   const float* cos_t; const float* sin_t;   /* [max_t][p_t]   */
   const float* cos_h; const float* sin_h;   /* [frame_h][p_h] */
   const float* cos_w; const float* sin_w;   /* [frame_w][p_w] */
   int32_t max_t, frame_h, frame_w, head_dim;
+  const float* cs_tok;                      /* [frame_h][frame_w][head_dim/2][2] or NULL */
 } cva_rope_tables;
 
 /* Frame cache of one attention layer (host struct holding device pointers).
@@ -155,6 +161,11 @@ int cva_rope_axis_pairs(int32_t head_dim, int32_t* p_t, int32_t* p_h, int32_t* p
  * [frame_w][p_w]. The caller copies them to the device once. */
 int cva_rope3d_precompute(const cva_rope_cfg* cfg, float* cos_t, float* sin_t,
                           float* cos_h, float* sin_h, float* cos_w, float* sin_w);
+
+/* Fills the HOST buffer cs_tok [frame_h][frame_w][head_dim/2][2] with the
+ * (cos, sin) of every spatial pair at every (h, w) position, the same floats
+ * as the per-axis tables, and (1, 0) for the temporal pairs. */
+int cva_rope3d_precompute_tokens(const cva_rope_cfg* cfg, float* cs_tok);
 
 /* ---- 1. rotary embedding with a global time index (section 2B) ----------- */
 

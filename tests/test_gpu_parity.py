@@ -626,6 +626,20 @@ def test_c3_topp_end_to_end_sampled(ops):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
+@pytest.mark.parametrize("key", ["c1s", "r64", "r128"])
+def test_chunk_call_writes_frame_means(ops, key):
+    # the fused call computes the new frames' frame means in the attention
+    # launch: equal to the token means of the stored keys
+    wl = WORKLOADS[key]
+    _, cache = _gpu_stream(ops, wl, wl.chunk)
+    kc = bits_to_f64(from_dev(cache.k))
+    got = cache.kpool_frm.cpu().numpy().astype(np.float64)
+    for f in range(wl.Fc):
+        slot = (wl.t0 + f) % wl.window
+        want = o_hsa.frame_mean(kc[:, :, slot, :wl.T_f])
+        np.testing.assert_allclose(got[:, :, slot], want, rtol=0, atol=2e-6 * max(1.0, np.abs(want).max()))
+
+
 # ---- denoising steps of a chunk -----------------------------------------------------------
 
 def test_denoising_passes_leave_no_trace(ops):
