@@ -382,6 +382,7 @@ int cva_rope3d_apply(const void* x, void* y, const cva_rope_tables* tables, cons
   a.job[0] = {static_cast<const uint16_t*>(x), kTokenMajor, static_cast<uint16_t*>(y),
               out_layout == 0 ? (int)kTokenMajor : (int)kHeadMajor, 1, nullptr, kPoolNone};
   a.njobs = 1;
+  a.err = device_error_word();
   a.tab = make_tab(tables, d.D);
   a.d = d;
   a.t0 = t0;
@@ -408,6 +409,7 @@ int cva_kv_append(const void* k, const void* v, const cva_kv_cache* cache,
   a.job[1] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
               kCacheSlots, 0, nullptr, kPoolNone};
   a.njobs = 2;
+  a.err = device_error_word();
   if (tables) a.tab = make_tab(tables, d.D);
   else axis_pairs(d.D, &a.tab.pt, &a.tab.ph, &a.tab.pw);
   a.d = d;
@@ -484,6 +486,7 @@ int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk
   a.job[0] = {static_cast<const uint16_t*>(q_rot), kHeadMajor, nullptr, kHeadMajor, 0, qpool_blk,
               kPoolChunk};
   a.njobs = 1;
+  a.err = device_error_word();
   axis_pairs(d.D, &a.tab.pt, &a.tab.ph, &a.tab.pw);
   a.d = d;
   a.t0 = 0;
@@ -822,6 +825,7 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
   a.job[2] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
               kCacheSlots, 0, nullptr, kPoolNone};
   a.njobs = 3;
+  a.err = device_error_word();
   a.tab = make_tab(tables, d.D);
   a.d = d;
   a.t0 = t0;

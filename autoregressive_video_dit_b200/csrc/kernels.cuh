@@ -22,6 +22,7 @@ struct StreamJob {
 struct RopePoolArgs {
   StreamJob job[3];
   int njobs;
+  int* err;      // device error word (bounded waits of the staged kernel)
   RopeTab tab;
   Dims d;
   int t0;
@@ -95,6 +96,10 @@ cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* c
 // Tiled TMA descriptor of a bf16 tensor [d2][d1][d0] (d0 innermost) with a
 // box of 64 x box1 elements and 128-byte swizzle (attn_sm100.cu).
 bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
+// Tiled TMA descriptor of a 2D bf16 (or fp32) tensor [d1][d0] with rows of
+// row_bytes, a box of box0 x box1 elements and no swizzle (attn_sm100.cu).
+bool make_map_2d(CUtensorMap* map, const void* base, bool fp32, uint64_t d0, uint64_t d1,
+                 uint64_t row_bytes, uint32_t box0, uint32_t box1);
 
 // ---- QKV projection + Causal-RoPE + append + block pooling (qkv_rope.cu) --
 struct QkvArgs {
