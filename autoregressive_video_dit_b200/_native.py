@@ -99,6 +99,7 @@ _SIGS = {
                                            c_void_p, c_void_p, c_void_p]),
     "cva_chunk_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables),
                                               c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
+    "cva_copy_rows_2d": (c_int32, [c_void_p, c_void_p] + [ctypes.c_int64] * 7 + [c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
     "cva_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
     "cva_kv_cache_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
@@ -375,6 +376,12 @@ def chunk_attention_topp(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables
     check(lib.cva_chunk_attention_topp(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
                                        ctypes.byref(tables.struct), t0, k_f, k_cap, p, _ptr(workspace),
                                        ws_bytes, _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def copy_rows_2d(src, dst, n0: int, n1: int, inner_bytes: int, src_strides, dst_strides, stream=None) -> None:
+    """Batched row copies over an n0 x n1 index space (byte strides; see cva.h)."""
+    check(lib.cva_copy_rows_2d(_ptr(src), _ptr(dst), n0, n1, inner_bytes, src_strides[0], src_strides[1],
+                               dst_strides[0], dst_strides[1], _stream(stream)))
 
 
 def chunk_attention_noalloc(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, k_f: int,

@@ -710,6 +710,21 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   return CVA_OK;
 }
 
+int cva_copy_rows_2d(const void* src, void* dst, int64_t n0, int64_t n1, int64_t inner_bytes,
+                     int64_t src_stride0, int64_t src_stride1, int64_t dst_stride0, int64_t dst_stride1,
+                     cva_stream_t stream) {
+  if (n0 < 0 || n1 < 0 || inner_bytes < 0) return fail(CVA_EINVAL, "negative size");
+  if (n0 == 0 || n1 == 0 || inner_bytes == 0) return CVA_OK;
+  if (!src || !dst) return fail(CVA_EINVAL, "NULL buffer");
+  const int64_t v[5] = {inner_bytes, src_stride0, src_stride1, dst_stride0, dst_stride1};
+  for (int i = 0; i < 5; ++i)
+    if (v[i] % 16) return fail(CVA_EINVAL, "sizes and strides must be multiples of 16 bytes");
+  if (!aligned(src, 16) || !aligned(dst, 16)) return fail(CVA_EINVAL, "src and dst must be 16-byte aligned");
+  RowCopy2D c = {n0, n1, inner_bytes, src_stride0, src_stride1, dst_stride0, dst_stride1};
+  cudaError_t e = launch_copy_rows_2d(src, dst, c, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "copy_rows_2d launch");
+}
+
 int cva_cag_noise_densities(int32_t n_chunks, int32_t Fc, int32_t window, int32_t blocks_per_frame,
                             double s_base, double s_target, double* densities) {
   if (!densities) return fail(CVA_EINVAL, "densities is NULL");

@@ -101,6 +101,14 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
 bool make_map_2d(CUtensorMap* map, const void* base, bool fp32, uint64_t d0, uint64_t d1,
                  uint64_t row_bytes, uint32_t box0, uint32_t box1);
 
+// ---- head-sharded path: batched row copies (shard.cu) -------------------
+struct RowCopy2D {
+  int64_t n0, n1, inner;    // rows i0 < n0, i1 < n1 of `inner` bytes
+  int64_t ss0, ss1;         // source strides (bytes)
+  int64_t ds0, ds1;         // destination strides (bytes)
+};
+cudaError_t launch_copy_rows_2d(const void* src, void* dst, const RowCopy2D& c, cudaStream_t stream);
+
 // ---- QKV projection + Causal-RoPE + append + block pooling (qkv_rope.cu) --
 struct QkvArgs {
   Dims d;

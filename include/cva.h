@@ -317,6 +317,24 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden,
                             int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
                             size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
+/* ---- head-sharded path (several GPUs) -------------------------------------
+ * "Accelerating Video Generation Inference with Sequential-Parallel 3D
+ * Positional Encoding Using a Global Time Index", section 2A: with the chunk
+ * sharded by tokens across G ranks, one all-to-all before the attention
+ * hands every rank all tokens of H/G heads, and one after it gives the
+ * token slices back. The exchange itself is the caller's collective (NCCL);
+ * this is the layout step around it.
+ *
+ * For i0 < n0 and i1 < n1 copies inner_bytes from src + i0*src_stride0 +
+ * i1*src_stride1 to dst + i0*dst_stride0 + i1*dst_stride1 (device memory,
+ * byte strides). Every size and stride a multiple of 16 and both pointers
+ * 16-byte aligned, else CVA_EINVAL; destination rows must not overlap each
+ * other or the source. Swapping the two outer dimensions of an
+ * [n0][n1][row] array is (ss0, ss1, ds0, ds1) = (n1*row, row, row, n0*row). */
+int cva_copy_rows_2d(const void* src, void* dst, int64_t n0, int64_t n1, int64_t inner_bytes,
+                     int64_t src_stride0, int64_t src_stride1, int64_t dst_stride0, int64_t dst_stride1,
+                     cva_stream_t stream);
+
 /* The fused chunk call without a caller workspace (the pages have no
  * counterpart; this exists for callers that cannot allocate device memory
  * when they call, such as a plugin whose host runtime owns every allocation
