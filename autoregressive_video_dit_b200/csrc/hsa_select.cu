@@ -81,6 +81,7 @@ __device__ __forceinline__ int rank_of(const uint64_t* key, int n, int i) {
   const uint64_t x = key[i];
   const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(key);
   int r = 0;
+#pragma unroll 8
   for (int j = 0; j < (n + 1) >> 1; ++j) {
     const ulonglong2 y = k2[j];
     r += (y.x > x ? 1 : 0) + (y.y > x ? 1 : 0);
