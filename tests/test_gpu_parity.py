@@ -123,6 +123,33 @@ def test_rope3d_apply(ops, key):
         assert np.all(hm[:, :, :, wl.T_f:] == 0)
 
 
+@pytest.mark.parametrize("key", ["c1", "r64", "r64s"])
+def test_rope_without_the_position_table(ops, key):
+    # tables without the per-position expansion take the per-pair lookup kernel:
+    # same results as with it
+    import torch
+    wl = WORKLOADS[key]
+    x = inputs(wl, wl.chunk)
+    tabs = _tables(ops, wl)
+    shp = shape_of(wl)
+    xd = to_dev(x["q"])
+    y_tok = torch.empty_like(xd)
+    ops.rope3d_apply(xd, y_tok, tabs, shp, wl.t0, 0)
+    tabs.struct.cs_tok = None
+    y_plain = torch.empty_like(xd)
+    ops.rope3d_apply(xd, y_plain, tabs, shp, wl.t0, 0)
+    cache = ops.DeviceKVCache(shp, wl.window)
+    ops.kv_append(to_dev(x["k"]), to_dev(x["v"]), cache, tabs, wl.t0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(from_dev(y_plain), from_dev(y_tok))
+    want = o_rope.rope_chunk(bits_to_f64(x["k"]), wl.Fh, wl.Fw, wl.Fc, wl.t0)
+    kc = bits_to_f64(from_dev(cache.k))
+    for f in range(wl.Fc):
+        got = kc[:, :, (wl.t0 + f) % wl.window, :wl.T_f]
+        w = np.transpose(want[:, f * wl.T_f:(f + 1) * wl.T_f], (0, 2, 1, 3))
+        assert np.all(np.abs(got - w) <= rope_tol(w))
+
+
 # ---- step 2 (+ K pooling): append ------------------------------------------------------
 
 @pytest.mark.parametrize("key", SMALL)
