@@ -56,6 +56,39 @@ def test_rope_tables_match_oracle(ops, D):
     assert ops.rope_axis_pairs(D) == o_rope.axis_split(D)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_position_table_repeats_the_axis_tables(ops, D):
+    # the per-position expansion holds exactly the per-axis floats, (1, 0) for
+    # the temporal pairs, and its pairs rotate like the oracle's angles
+    Fh, Fw = 7, 11
+    t = ops.rope3d_precompute(D, 8, Fh, Fw)
+    tok = t["cs_tok"]
+    pt, ph, pw = ops.rope_axis_pairs(D)
+    assert tok.shape == (Fh, Fw, D // 2, 2)
+    np.testing.assert_array_equal(tok[:, :, :pt, 0], 1.0)
+    np.testing.assert_array_equal(tok[:, :, :pt, 1], 0.0)
+    for h in range(Fh):
+        for w in range(Fw):
+            np.testing.assert_array_equal(tok[h, w, pt:pt + ph, 0], t["cos_h"][h])
+            np.testing.assert_array_equal(tok[h, w, pt:pt + ph, 1], t["sin_h"][h])
+            np.testing.assert_array_equal(tok[h, w, pt + ph:, 0], t["cos_w"][w])
+            np.testing.assert_array_equal(tok[h, w, pt + ph:, 1], t["sin_w"][w])
+    ang = o_rope.pair_angles(D, np.zeros(Fh * Fw), np.repeat(np.arange(Fh), Fw), np.tile(np.arange(Fw), Fh))
+    np.testing.assert_allclose(tok[..., 0].reshape(Fh * Fw, -1), np.cos(ang), rtol=0, atol=6e-8)
+    np.testing.assert_allclose(tok[..., 1].reshape(Fh * Fw, -1), np.sin(ang), rtol=0, atol=6e-8)
+
+
+def test_copy_rows_2d_validates_before_launching(ops):
+    fake = ctypes.c_void_p(1 << 41)
+    f = ops.lib.cva_copy_rows_2d
+    assert f(fake, fake, 0, 4, 16, 16, 16, 16, 16, None) == 0           # nothing to copy
+    assert f(fake, fake, 2, 2, 24, 48, 24, 24, 48, None) == ops.CVA_EINVAL  # 24-byte rows
+    assert f(fake, fake, 2, 2, 32, 40, 32, 32, 64, None) == ops.CVA_EINVAL  # stride not 16-aligned
+    assert f(ctypes.c_void_p((1 << 41) + 8), fake, 2, 2, 32, 64, 32, 32, 64, None) == ops.CVA_EINVAL
+    assert f(None, fake, 2, 2, 32, 64, 32, 32, 64, None) == ops.CVA_EINVAL
+    assert f(fake, fake, -1, 2, 32, 64, 32, 32, 64, None) == ops.CVA_EINVAL
+
+
 def _lib_budget(ops, wl, chunk, hist):
     return ops.cag_budget(chunk, hist, wl.nb, dense=wl.dense, k_f_max=wl.k_f_max,
                           d_base=(wl.d_base.numerator, wl.d_base.denominator),
