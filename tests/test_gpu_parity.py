@@ -261,6 +261,25 @@ def test_hsa_select_staged_c3_full_size(ops, chunk):
     assert bad == 0 and near <= 0.02 * n, (bad, near, n)
 
 
+def _max_history_workload(k_b):
+    # 256 history frames (the selection's limit) of 16x16 tokens in 4 blocks:
+    # the second level ranks 1024 candidates (its limit), k_b of them kept
+    return WORKLOADS["c1s"].replace(H=1, D=64, Fh=16, Fw=16, window=259, chunk=87, k_f_max=256,
+                                    k_b_fixed=k_b)
+
+
+@pytest.mark.parametrize("k_b", [700, 1024])
+def test_select_and_attention_at_the_size_limits(ops, k_b):
+    wl = _max_history_workload(k_b)
+    run = _oracle_run(wl, wl.chunk)
+    assert run["k_f"] == 256 and run["k_b"] == k_b and len(run["hist"]) == 86
+    assert run["frames"].shape[-1] == 256 and run["blocks"].shape[-1] == k_b
+    _, _, fi, bi, bc = _staged_select(ops, wl, run)
+    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    assert bad == 0 and near <= 0.1 * n, (bad, near, n)
+    _check_attention(ops, wl, run, run["blocks"], split=True)
+
+
 # ---- step 5: attention ------------------------------------------------------------------
 
 def _check_attention(ops, wl, run, blocks, rows=None, t_begin=0, split=False):
