@@ -287,7 +287,12 @@ int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden,
 /* ---- fused chunk call ---------------------------------------------------- */
 
 /* Steps 1-5 for one chunk: RoPE(Q) with Q pooling, RoPE(K)+append+K pooling,
- * selection with (k_f, k_b) (dense when k_f < 0), attention.
+ * selection with (k_f, k_b) (dense when k_f < 0), attention. The launches,
+ * in stream order: the rotate/append/pool kernel (Q, K and V in one pass),
+ * the selection (sparse only), the attention (whose spare warps also write
+ * the frame means of the new cache frames), the merge of split tail tiles
+ * (only when the query tiles leave a partial wave). Results equal the staged
+ * calls' up to fp32 rounding order.
  *   q, k, v: bf16 [B, Lq, H, D]; out: bf16 [B, Lq, H, D]; lse: fp32
  *   [B][H][Lq] or NULL. workspace: cva_chunk_workspace_bytes() bytes. */
 int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b,
