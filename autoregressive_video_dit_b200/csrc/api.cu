@@ -127,7 +127,7 @@ void history(const cva_kv_cache* c, int t0, int* t_lo, int* F) {
 }
 
 struct ChunkWs {
-  size_t q_rot, qpool, frame_idx, block_idx, block_cnt, attn, total;
+  size_t q_rot, qpool, frame_idx, block_idx, block_cnt, qpair, attn, total;
 };
 
 // Attention scratch: partial (O, max, sum) of the pieces of split tail tiles.
@@ -144,6 +144,7 @@ ChunkWs chunk_ws_layout(const Dims& d, int k_f, int k_b) {
   w.frame_idx = off; off += round256(bhq * (size_t)(k_f > 0 ? k_f : 0) * 4);
   w.block_idx = off; off += round256(bhq * (size_t)(k_b > 0 ? k_b : 0) * 4);
   w.block_cnt = off; off += round256(bhq * 4);
+  w.qpair = off; off += round256((size_t)d.B * d.H * ((d.Fc * d.T_pad + 127) / 128) * 2 * 4);
   w.attn = off; off += attn_split_bytes(d);
   w.total = off;
   return w;
@@ -592,11 +593,34 @@ static int sm_count() {
   return counts[dev];
 }
 
+// Tiles of two 64-row query blocks paired by their picked frames (the fused
+// calls with a selection); *qpair stays NULL when blocks are 128 rows (one
+// block per tile), when fewer than 2 k_f history frames leave little to pair,
+// or beyond the pairing's limits (tiles then hold blocks 2m and 2m+1).
+static int pair_impl(const Dims& d, const cva_kv_cache* cache, int t0, int k_f, const int32_t* fidx,
+                     int32_t* qpair_ws, const int32_t** qpair, cudaStream_t s) {
+  *qpair = nullptr;
+  if (d.blk != 64) return CVA_OK;
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
+  const int kfe = k_f < F ? k_f : F;
+  // Pairs pay off only when the query blocks' frame picks can differ much:
+  // with at least twice as many history frames as picks.
+  if (F == 0 || kfe < 1 || F < 2 * kfe) return CVA_OK;
+  const int MT = (d.Fc * d.T_pad + 127) / 128;
+  cudaError_t e = launch_pair_query_blocks(fidx, kfe, d, t_lo, F, MT, qpair_ws, s);
+  if (e == cudaErrorInvalidValue) return CVA_OK;  // beyond the pairing's limits: default tiles
+  if (e != cudaSuccess) return cuda_fail(e, "pair_query_blocks launch");
+  *qpair = qpair_ws;
+  return CVA_OK;
+}
+
 // frame_means: the launch also writes the frame means of the chunk's cache
 // frames (its spare warps), from the block means the chunk's append wrote.
 static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const int32_t* block_idx,
                      const int32_t* block_cnt, int k_b_max, void* out, float* lse, void* split_ws,
-                     size_t split_bytes, cudaStream_t s, bool frame_means = false) {
+                     size_t split_bytes, cudaStream_t s, bool frame_means = false,
+                     const int32_t* qpair = nullptr) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -620,6 +644,7 @@ static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const
     a.kpool_blk = cache->kpool_blk;
     a.kpool_frm = cache->kpool_frm;
   }
+  a.qpair = qpair;
   // Tail split: the tiles of the last, partial wave are cut into key-range
   // pieces so that they fill the SMs (needs the scratch; else unsplit).
   const int tiles = a.MT * d.B * d.H;
@@ -698,13 +723,16 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   rc = qkv_rope_append_impl(x, w_qkv, hidden, cache, tables, t0, q_rot, sparse ? qpool : nullptr, stream, false);
   if (rc) return rc;
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
+  const int32_t* qpair = nullptr;
   if (sparse) {
     rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, 0.f, s);
+    if (rc) return rc;
+    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;
@@ -853,14 +881,17 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
 
   // step 4
   const bool sparse = !dense && F > 0;
+  const int32_t* qpair = nullptr;
   if (sparse) {
     rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, topp, s);
+    if (rc) return rc;
+    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   // step 5 (with the frame means of the new cache frames)
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;

@@ -146,6 +146,17 @@ struct Stream {
   }
 };
 
+// Query block in rows [64 half, 64 half + 64) of tile m of head bh (64-row blocks).
+__device__ __forceinline__ int tile_qb(const AttnArgs& a, int bh, int m, int half) {
+  return a.qpair ? a.qpair[((size_t)bh * a.MT + m) * 2 + half] : 2 * m + half;
+}
+// Row of the padded chunk held in row r of tile m (-1: none).
+__device__ __forceinline__ int tile_row(const AttnArgs& a, int bh, int m, int r) {
+  if (!a.qpair) return m * kBM + r;
+  const int qb = a.qpair[((size_t)bh * a.MT + m) * 2 + (r >> 6)];
+  return qb < 0 ? -1 : qb * 64 + (r & 63);
+}
+
 // Builds the key stream of the CTA's lanes (tile m0 and, if has_b, m0 + 1)
 // into `ents`; must be called by all threads of the CTA.
 __device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, uint32_t* ents,
@@ -166,8 +177,8 @@ __device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, ui
     const int nq = (d.blk == 64) ? 2 : 1;
     for (int x = 0; x < (has_b ? 2 : 1); ++x) {
       for (int q = 0; q < nq; ++q) {
-        const int qb = (d.blk == 64) ? 2 * (m0 + x) + q : m0 + x;
-        if (qb >= d.NQB) continue;
+        const int qb = (d.blk == 64) ? tile_qb(a, bh, m0 + x, q) : m0 + x;
+        if (qb < 0 || qb >= d.NQB) continue;
         const size_t u = (size_t)bh * d.NQB + qb;
         int c = a.block_cnt ? a.block_cnt[u] : a.k_b_max;
         if (c < 0 || c > a.k_b_max) {
@@ -378,9 +389,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       };
       if (N > 0) {
+        // the tile's two 64-row halves (a half with no query block reads past
+        // the chunk's rows: zero fill)
+        const int q0 = tile_row(a, bh, m, 0), q1 = tile_row(a, bh, m, 64);
+        const int past = a.d.Fc * a.d.T_pad;
         mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, m * kBM, bh);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, q0 < 0 ? past : q0, bh);
+          tma_load_3d(smem + L::kQ + c * L::kChunkBytes + 8192, &tmQ, &bar[kBarQ], c * 64, q1 < 0 ? past : q1, bh);
+        }
       }
       // Tile t goes to slot t mod 2 once the tile before it there (t - 2)
       // was consumed; K and V advance independently.
@@ -592,9 +609,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         if (par == 0) reinterpret_cast<float2*>(a.part_ml)[(size_t)slot * kBM + r] = make_float2(M, l_tot);
       } else {
-        const int pr = m * kBM + r;  // row in the padded chunk
-        const int f = pr / d.T_pad;
-        const int rr = pr - f * d.T_pad;
+        const int pr = tile_row(a, bh, m, r);  // row in the padded chunk, or -1
+        const int f = pr < 0 ? d.Fc : pr / d.T_pad;
+        const int rr = pr < 0 ? 0 : pr - f * d.T_pad;
         const bool row_ok = (f < d.Fc) && (rr < d.T_f);
         const int bb = bh / d.H;
         const int h = bh - bb * d.H;
@@ -683,7 +700,8 @@ __global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a) {
     acc.z += w * o.z;
     acc.w += w * o.w;
   }
-  const int pr = m * kBM + r;
+  const int pr = tile_row(a, bh, m, r);
+  if (pr < 0) return;
   const int f = pr / d.T_pad;
   const int rr = pr - f * d.T_pad;
   if (f >= d.Fc || rr >= d.T_f) return;
@@ -765,7 +783,7 @@ cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* c
   const Dims& d = a.d;
   CUtensorMap mq, mk, mv;
   const uint64_t bh = (uint64_t)d.B * d.H;
-  if (!make_map(&mq, q_rot, d.D, (uint64_t)d.Fc * d.T_pad, bh, 128) ||
+  if (!make_map(&mq, q_rot, d.D, (uint64_t)d.Fc * d.T_pad, bh, 64) ||
       !make_map(&mk, cache_k, d.D, (uint64_t)a.W * d.T_pad, bh, 64) ||
       !make_map(&mv, cache_v, d.D, (uint64_t)a.W * d.T_pad, bh, 64)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point or tensor shape)";

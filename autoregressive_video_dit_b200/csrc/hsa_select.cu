@@ -260,6 +260,93 @@ __global__ void __launch_bounds__(kSelThreads) hsa_select_kernel(SelectArgs a, i
   if (tid == 0 && a.block_cnt) a.block_cnt[u] = nout;
 }
 
+// ---- pairing of 64-row query blocks into 128-row attention tiles -----------
+//
+// A tile of two query blocks iterates the union of their block lists, so the
+// pairs are chosen by the frames the blocks picked. One CTA per
+// (batch*head): its threads tabulate the number of picked frames every two
+// query blocks share; then one warp walks the query blocks in order and pairs
+// each unpaired one with the unpaired block after it that shares the most
+// frames, ties to the lower index (one packed max-reduction per step); a
+// block left over pairs with none (-1). Pair n becomes tile n.
+constexpr int kPairMaxQB = 128;
+constexpr int kPairWords = kSelMaxFrames / 32;
+constexpr int kPairThreads = 256;
+
+__global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const int32_t* __restrict__ frame_idx,
+                                                                         int kfe, int NQB, int t_lo, int MT,
+                                                                         int32_t* qpair) {
+  __shared__ uint32_t mask[kPairMaxQB][kPairWords];
+  __shared__ uint8_t ov[kPairMaxQB][kPairMaxQB];
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x;
+  for (int qb = tid; qb < NQB; qb += kPairThreads) {  // one thread per query block: no write races
+#pragma unroll
+    for (int k = 0; k < kPairWords; ++k) mask[qb][k] = 0u;
+    const int32_t* fr = frame_idx + ((size_t)bh * NQB + qb) * kfe;
+    for (int i = 0; i < kfe; ++i) {
+      const int p = fr[i] - t_lo;  // position in the history, < 256
+      if (p >= 0 && p < kSelMaxFrames) mask[qb][p >> 5] |= 1u << (p & 31);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NQB * NQB; e += kPairThreads) {
+    const int i = e / NQB, j = e - (e / NQB) * NQB;
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < kPairWords; ++k) c += __popc(mask[i][k] & mask[j][k]);
+    ov[i][j] = (uint8_t)c;  // shared frames, at most kfe <= 255
+  }
+  __syncthreads();
+  if (tid >= 32) return;
+  const int lane = tid;
+  int32_t* out = qpair + (size_t)bh * MT * 2;
+  uint32_t tk[kPairMaxQB / 32] = {};  // taken query blocks, the same in every lane
+  int n = 0;
+  // bit i of tk, and setting it, without indexing the array at run time (registers)
+  auto bit = [&](int i) {
+    uint32_t w = 0u;
+#pragma unroll
+    for (int k = 0; k < kPairMaxQB / 32; ++k) w = (i >> 5) == k ? tk[k] : w;
+    return (w >> (i & 31)) & 1u;
+  };
+  auto set = [&](int i) {
+#pragma unroll
+    for (int k = 0; k < kPairMaxQB / 32; ++k)
+      if ((i >> 5) == k) tk[k] |= 1u << (i & 31);
+  };
+  for (int i = 0; i < NQB; ++i) {
+    if (bit(i)) continue;
+    // key: shared frames + 1, then the complement of j (ties to the lower j); 0: none
+    unsigned key = 0u;
+#pragma unroll
+    for (int k = 0; k < kPairMaxQB / 32; ++k) {
+      const int j = 32 * k + lane;
+      if (j > i && j < NQB && !((tk[k] >> lane) & 1u)) key = max(key, (1u + ov[i][j]) << 16 | (0xFFFFu - (unsigned)j));
+    }
+    key = __reduce_max_sync(0xFFFFFFFFu, key);
+    const int best = key ? (int)(0xFFFFu - (key & 0xFFFFu)) : -1;
+    set(i);
+    if (best >= 0) set(best);
+    if (lane == 0) {
+      out[2 * n] = i;
+      out[2 * n + 1] = best;
+    }
+    ++n;
+  }
+  for (int t = n + lane; t < MT; t += 32) {  // tiles without query blocks (none when MT = ceil(NQB / 2))
+    out[2 * t] = -1;
+    out[2 * t + 1] = -1;
+  }
+}
+
+cudaError_t launch_pair_query_blocks(const int32_t* frame_idx, int kfe, const Dims& d, int t_lo, int F, int MT,
+                                     int32_t* qpair, cudaStream_t stream) {
+  if (d.NQB > kPairMaxQB || F > kSelMaxFrames || kfe < 1 || kfe > 255) return cudaErrorInvalidValue;
+  pair_query_blocks_kernel<<<d.B * d.H, kPairThreads, 0, stream>>>(frame_idx, kfe, d.NQB, t_lo, MT, qpair);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   const int kfe = a.k_f < a.F ? a.k_f : a.F;
   const int nmax = a.F > kfe * a.d.nb ? a.F : kfe * a.d.nb;

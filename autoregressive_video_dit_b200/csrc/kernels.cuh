@@ -60,6 +60,10 @@ struct SelectArgs {
   float temp_log2;         // log2(e) / sqrt(D)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+// Pairs each head's 64-row query blocks into 128-row attention tiles by the
+// overlap of their picked frames (hsa_select.cu).
+cudaError_t launch_pair_query_blocks(const int32_t* frame_idx, int kfe, const Dims& d, int t_lo, int F,
+                                     int MT, int32_t* qpair, cudaStream_t stream);
 
 // ---- step 5: attention (attn_sm100.cu) -----------------------------------
 struct AttnArgs {
@@ -79,6 +83,10 @@ struct AttnArgs {
   int Qf, pieces;
   float* part_o;             // [piece slot][128][D] fp32, unnormalised
   float* part_ml;            // [piece slot][128][2] running max (log2 units), sum
+  // Query blocks held by each 128-row tile when blocks are 64 rows:
+  // [B*H][MT][2] (rows 0-63, rows 64-127; -1 for none), or nullptr for the
+  // blocks 2m and 2m+1 of tile m.
+  const int32_t* qpair;
   // Optional: frame means of the chunk's cache frames (t0 .. t0+Fc-1) from
   // their block means, computed by the CTAs' spare warps.
   const float* kpool_blk;    // [B][H][W][nb][D]

@@ -536,7 +536,10 @@ def run_cuda(args):
                          "achieved": rb / (rope_avg * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": rb / (rope_avg * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
                          "algorithmic_bytes": rb},
-        "gpu_launches": n * (1 + (1 if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
+        # rotate/append/pool; selection and (64-row blocks, history of at least 2 k_f frames)
+        # query-block pairing; attention (+ merge)
+        "gpu_launches": n * (1 + ((1 + (wl.blk == 64 and st["F"] >= 2 * min(st["k_f"], st["F"])))
+                                  if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
         "clocks": clocks,
     }
     if e2e:

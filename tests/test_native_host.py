@@ -219,8 +219,9 @@ def test_workspace_bytes(ops):
     bhq = wl.B * wl.H * wl.NQB
     # attention scratch: partial O, max and sum of up to 160 key-range pieces
     attn = r(160 * 128 * wl.D * 4) + r(160 * 128 * 2 * 4)
+    MT = -(-wl.Fc * wl.T_pad // 128)   # 128-row query tiles per head; a pair of query blocks each
     want = (r(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r(bhq * wl.D * 4) + r(bhq * 8 * 4)
-            + r(bhq * 120 * 4) + r(bhq * 4) + attn)
+            + r(bhq * 120 * 4) + r(bhq * 4) + r(wl.B * wl.H * MT * 2 * 4) + attn)
     assert ops.chunk_workspace_bytes(s, 8, 120) == want
     assert ops.attn_workspace_bytes(s, 120) == attn
 
