@@ -11,15 +11,16 @@
 // One CTA handles one (batch*head, frame, block) of up to three tensors
 // (Q, K, V) in a single pass over HBM. Each thread owns 8 consecutive
 // elements (one 16-byte vector) of a row, so a warp reads and writes whole
-// rows; a thread issues the loads of its rows of a batch, for all tensors,
-// together with its 32-byte entries of the per-position (cos, sin) table,
-// before it uses any of them. The job
-// properties (which tensors are rotated or pooled) are template parameters,
-// so the per-row work is the loads, the rotation, the pooling sums and the
-// stores. Block sums are reduced in a fixed order from the bf16 values
-// actually stored (deterministic). Frame means of the block means are a
-// separate step (frame_pool_kernel, or the attention kernel's spare warps
-// in the fused chunk call).
+// rows. rope_pool_tma_kernel (below) stages the block's rows and its rows of
+// the per-position (cos, sin) table in shared memory through TMA;
+// rope_pool_kernel, for tables without the per-position expansion, loads a
+// batch of rows into registers and looks every pair up in the per-axis
+// tables. The job properties (which tensors are rotated or pooled) are
+// template parameters, so the per-row work is the loads, the rotation, the
+// pooling sums and the stores. Block sums are reduced in a fixed order from
+// the bf16 values actually stored (deterministic). Frame means of the block
+// means are a separate step (frame_pool_kernel, or the attention kernel's
+// spare warps in the fused chunk call).
 #include "kernels.cuh"
 
 namespace cva {
