@@ -221,6 +221,16 @@ int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream)
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "exp2_poly_eval launch");
 }
 
+int cva_diag_wait_timeout(int32_t limit_us, int32_t* result, cva_stream_t stream) {
+  if (!result) return fail(CVA_EINVAL, "result is NULL");
+  if (!aligned(result, 4)) return fail(CVA_EINVAL, "result must be 4-byte aligned");
+  if (limit_us < 1 || limit_us > 1000000) return fail(CVA_EINVAL, "limit_us must lie in [1, 1000000]");
+  int* err = device_error_word();
+  if (!err) return fail(CVA_ELAUNCH, "device error word unavailable");
+  cudaError_t e = launch_wait_timeout(err, result, (uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "diag_wait_timeout launch");
+}
+
 int cva_rope_axis_pairs(int32_t head_dim, int32_t* p_t, int32_t* p_h, int32_t* p_w) {
   if (!p_t || !p_h || !p_w) return fail(CVA_EINVAL, "NULL output");
   if (head_dim < 6 || head_dim % 2) return fail(CVA_EINVAL, "head_dim must be even and >= 6");
@@ -820,24 +830,21 @@ int cva_chunk_workspace_bytes(const cva_shape* shape, int32_t k_f, int32_t k_b, 
 
 }  // extern "C"
 
-// Steps 1-5 from q, k, v; topp > 0 selects blocks by the top-p budget with
-// cap k_b.
-static int chunk_attention_impl(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
-                                const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
-                                float topp, void* workspace, size_t ws_bytes, void* out, float* lse,
-                                cva_stream_t stream) {
+// Every host check of the fused chunk call except those of the workspace;
+// *ws_need gets the workspace bytes the call needs.
+int cva::check_chunk_call(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                          const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                          const void* out, size_t* ws_need) {
   int rc = check_cache(cache);
   if (rc) return rc;
-  if (!q || !k || !v || !out || !workspace) return fail(CVA_EINVAL, "NULL buffer");
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(workspace, 256))
-    return fail(CVA_EINVAL, "q, k, v, out must be 16-byte and workspace 256-byte aligned");
+  if (!q || !k || !v || !out) return fail(CVA_EINVAL, "NULL buffer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return fail(CVA_EINVAL, "q, k, v and out must be 16-byte aligned");
   if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
   const Dims d = make_dims(cache->shape);
   rc = check_tables(tables, d, t0);
   if (rc) return rc;
   const bool dense = k_f < 0;
-  const ChunkWs w = chunk_ws_layout(d, dense ? 0 : k_f, dense ? 0 : k_b);
-  if (ws_bytes < w.total) return fail(CVA_ENOMEM, "workspace %zu bytes < %zu needed", ws_bytes, w.total);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
   if (!dense) {
@@ -850,6 +857,27 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
   }
   rc = check_attn_limits(d, F, dense || F == 0, dense ? 0 : k_b);
   if (rc) return rc;
+  *ws_need = chunk_ws_layout(d, dense ? 0 : k_f, dense ? 0 : k_b).total;
+  return CVA_OK;
+}
+
+// Steps 1-5 from q, k, v; topp > 0 selects blocks by the top-p budget with
+// cap k_b.
+static int chunk_attention_impl(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                                const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                                float topp, void* workspace, size_t ws_bytes, void* out, float* lse,
+                                cva_stream_t stream) {
+  size_t need = 0;
+  int rc = check_chunk_call(q, k, v, cache, tables, t0, k_f, k_b, out, &need);
+  if (rc) return rc;
+  if (!workspace) return fail(CVA_EINVAL, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(CVA_EINVAL, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(CVA_ENOMEM, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  const Dims d = make_dims(cache->shape);
+  const bool dense = k_f < 0;
+  const ChunkWs w = chunk_ws_layout(d, dense ? 0 : k_f, dense ? 0 : k_b);
+  int t_lo, F;
+  history(cache, t0, &t_lo, &F);
 
   char* ws = static_cast<char*>(workspace);
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws + w.q_rot);

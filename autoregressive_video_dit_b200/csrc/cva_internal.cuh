@@ -144,14 +144,14 @@ __device__ __forceinline__ bool mbar_sleep(uint64_t* bar, uint32_t parity, uint3
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err) {
+                                          int* err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t_start = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t_start > kWaitLimitNs) {
+      if (globaltimer_ns() - t_start > limit_ns) {
         *abort_flag = 1;
         latch_error(err, CVA_DEV_TIMEOUT);
         return false;

@@ -138,7 +138,14 @@ cudaError_t launch_qkv_rope(const QkvArgs& a, const void* x, const void* w, cuda
 // Sets the thread-local message cva_last_error() returns; returns `code`.
 int report_error(int code, const char* msg);
 
+// Host checks of cva_chunk_attention's arguments other than the workspace
+// (same codes and messages); *ws_need gets the workspace bytes it needs.
+int check_chunk_call(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                     const cva_rope_tables* tables, int32_t t0, int32_t k_f, int32_t k_b,
+                     const void* out, size_t* ws_need);
+
 // ---- diagnostics (diag.cu) ------------------------------------------------
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+cudaError_t launch_wait_timeout(int* err, int* result, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace cva

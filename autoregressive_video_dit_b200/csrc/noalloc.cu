@@ -3,8 +3,13 @@
 // host runtime that owns every allocation and hands the plugin only its
 // input and output buffers, or a real-time loop that forbids allocation
 // after start-up. Instead of a caller-provided workspace it uses one fixed
-// scratch array in this file, reserved on every device that loads the
-// library for as long as the process lives.
+// scratch array in this file. Under CUDA's lazy module loading (the default)
+// the array is reserved on a device when this file's module is first loaded
+// there, which is the first call on that device (its cudaGetSymbolAddress);
+// from then on it stays reserved until the process exits. That first call can
+// therefore fail for lack of device memory, and it should be made during
+// start-up, before any stream capture (or load eagerly with
+// CUDA_MODULE_LOADING=EAGER, which reserves it when the library's modules load).
 #include <stdio.h>
 
 #include <mutex>
@@ -20,7 +25,8 @@ constexpr size_t kNoAllocScratchBytes = 64u << 20;  // 64 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // The array's name is only a host-side stand-in; its device address is
-// looked up once per device, with that device current, and cached.
+// looked up once per device, with that device current, and cached. The
+// lookup loads the module (and so reserves the array) on that device.
 void* noalloc_scratch_address(int* rc) {
   static std::mutex mu;
   static void* addr[128] = {};
@@ -53,9 +59,11 @@ extern "C" int cva_chunk_attention_noalloc(const void* q, const void* k, const v
                                            const cva_kv_cache* cache, const cva_rope_tables* tables,
                                            int32_t t0, int32_t k_f, int32_t k_b, void* out, float* lse,
                                            cva_stream_t stream) {
-  if (!cache) return cva::report_error(CVA_EINVAL, "cache is NULL");
+  // The arguments are checked first, exactly as cva_chunk_attention checks
+  // them (a budget beyond the candidates is CVA_ERANGE, not a size problem);
+  // then the scratch this shape and budget need is compared with the array.
   size_t need = 0;
-  int rc = cva_chunk_workspace_bytes(&cache->shape, k_f, k_b, &need);
+  int rc = cva::check_chunk_call(q, k, v, cache, tables, t0, k_f, k_b, out, &need);
   if (rc) return rc;
   if (need > kNoAllocScratchBytes) {
     char msg[256];

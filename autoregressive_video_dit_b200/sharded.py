@@ -118,19 +118,32 @@ class HeadShardedChunkAttention:
             self.cache = ops.DeviceKVCache(self.local_shape, window, t_begin, device=device)
             attend = self._attend_native
         self.attend = attend
+        # Buffers kept across calls (allocated on first use): the exchange
+        # buffers, the rank's whole-chunk Q, K, V and output of its heads, and
+        # the chunk workspace (grown when a larger budget needs more).
+        self._bufs = {}
+        self.ws = None
+
+    def _buf(self, name, numel, dtype, device):
+        import torch
+        t = self._bufs.get(name)
+        if t is None or t.numel() != numel or t.dtype != dtype or t.device != torch.device(device):
+            t = torch.empty(numel, dtype=dtype, device=device)
+            self._bufs[name] = t
+        return t
 
     def _attend_native(self, q, k, v, t0, k_f, k_b, out):
         import torch
         from . import _native as ops
-        ws = torch.empty(ops.chunk_workspace_bytes(self.local_shape, k_f, k_b), dtype=torch.uint8,
-                         device=q.device)
-        ops.chunk_attention(q, k, v, self.cache, self.tables, t0, k_f, k_b, ws, out)
+        need = ops.chunk_workspace_bytes(self.local_shape, k_f, k_b)
+        if self.ws is None or self.ws.numel() < need or self.ws.device != q.device:
+            self.ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ops.chunk_attention(q, k, v, self.cache, self.tables, t0, k_f, k_b, self.ws, out)
 
     def pack(self, q, k, v):
         """The rank's token slices of Q, K and V laid out for the exchange: [P][3][B][L][row]."""
-        import torch
         pl = self.plan
-        send = torch.empty(3 * pl.slab * pl.P // q.element_size(), dtype=q.dtype, device=q.device)
+        send = self._buf("send", 3 * pl.slab * pl.P // q.element_size(), q.dtype, q.device)
         for t, x in enumerate((q, k, v)):
             _apply(self.copy_rows, x.contiguous(), send, pl.pack(t))
         return send
@@ -138,15 +151,15 @@ class HeadShardedChunkAttention:
     def compute(self, recv, t0: int, k_f: int, k_b: int):
         """The path on this rank's heads from the exchanged Q, K and V; returns
         the output laid out for the exchange back: [P][B][L][row]."""
-        import torch
         pl = self.plan
         B, Hl, D = pl.B, pl.Hl, pl.D
-        loc = [torch.empty((B, pl.Lq, Hl, D), dtype=recv.dtype, device=recv.device) for _ in range(3)]
+        n = B * pl.Lq * Hl * D
+        loc = [self._buf(f"loc{t}", n, recv.dtype, recv.device).view(B, pl.Lq, Hl, D) for t in range(3)]
         for t in range(3):
             _apply(self.copy_rows, recv, loc[t], pl.unpack(t))
-        out_l = torch.empty((B, pl.Lq, Hl, D), dtype=recv.dtype, device=recv.device)
+        out_l = self._buf("out_l", n, recv.dtype, recv.device).view(B, pl.Lq, Hl, D)
         self.attend(loc[0], loc[1], loc[2], t0, k_f, k_b, out_l)
-        send2 = torch.empty(pl.slab * pl.P // recv.element_size(), dtype=recv.dtype, device=recv.device)
+        send2 = self._buf("send2", pl.slab * pl.P // recv.element_size(), recv.dtype, recv.device)
         _apply(self.copy_rows, out_l, send2, pl.pack_out())
         return send2
 
@@ -157,12 +170,11 @@ class HeadShardedChunkAttention:
         _apply(self.copy_rows, recv2, out, self.plan.unpack_out())
 
     def __call__(self, q, k, v, t0: int, k_f: int, k_b: int, out) -> None:
-        import torch
         import torch.distributed as dist
         send = self.pack(q, k, v)
-        recv = torch.empty_like(send)
+        recv = self._buf("recv", send.numel(), send.dtype, send.device)
         dist.all_to_all_single(recv, send, group=self.group)     # one exchange for Q, K and V
         send2 = self.compute(recv, t0, k_f, k_b)
-        recv2 = torch.empty_like(send2)
+        recv2 = self._buf("recv2", send2.numel(), send2.dtype, send2.device)
         dist.all_to_all_single(recv2, send2, group=self.group)
         self.finish(recv2, out)

@@ -184,7 +184,12 @@ int cva_rope3d_apply(const void* x, void* y, const cva_rope_tables* tables,
 
 /* ---- 2. cache append (+ K pooling of step 3) ----------------------------- */
 
-/* Writes the chunk's frames t0 .. t0+Fc-1 into their slots: K rotated (or
+/* "Accelerating Video Generation Inference with Sequential-Parallel 3D
+ * Positional Encoding Using a Global Time Index", section 1 (problem): the
+ * Self-Forcing style generator produces the video chunk by chunk, caching the
+ * keys and values of earlier chunks (KV caching) in a rolling window; the
+ * keys are cached already rotated with their global time index (section 2B).
+ * Writes the chunk's frames t0 .. t0+Fc-1 into their slots: K rotated (or
  * copied as is when tables == NULL, for keys rotated upstream), V copied,
  * pad rows zeroed, and the block-mean and frame-mean of the stored (bf16)
  * keys written to kpool_blk / kpool_frm in fp32.
@@ -193,7 +198,9 @@ int cva_rope3d_apply(const void* x, void* y, const cva_rope_tables* tables,
 int cva_kv_append(const void* k, const void* v, const cva_kv_cache* cache,
                   const cva_rope_tables* tables, int32_t t0, cva_stream_t stream);
 
-/* History frames a chunk at t0 sees: [max(t_begin, t0 + Fc - W), t0). */
+/* History frames a chunk at t0 sees: [max(t_begin, t0 + Fc - W), t0) -- the
+ * cached earlier frames still inside the rolling window of W frames (the same
+ * section 1 passage as cva_kv_append: KV caching with a rolling window). */
 int cva_history_frames(const cva_kv_cache* cache, int32_t t0, int32_t* t_lo,
                        int32_t* count);
 
@@ -286,7 +293,12 @@ int cva_qkv_rope_append(const void* x, const void* w_qkv, int32_t hidden,
 
 /* ---- fused chunk call ---------------------------------------------------- */
 
-/* Steps 1-5 for one chunk: RoPE(Q) with Q pooling, RoPE(K)+append+K pooling,
+/* Steps 1-5 for one chunk, in the order "Light Forcing" section 2.2 gives
+ * them (token compression by mean pooling, frame then block selection, then
+ * attention over the picked frame-block pairs) after the rotation with the
+ * global time index of "Accelerating Video Generation Inference with
+ * Sequential-Parallel 3D Positional Encoding Using a Global Time Index",
+ * section 2B: RoPE(Q) with Q pooling, RoPE(K)+append+K pooling,
  * selection with (k_f, k_b) (dense when k_f < 0), attention. The launches,
  * in stream order: the rotate/append/pool kernel (Q, K and V in one pass),
  * the selection (sparse only), the attention (whose spare warps also write
@@ -302,7 +314,9 @@ int cva_chunk_attention(const void* q, const void* k, const void* v,
                         int32_t t0, int32_t k_f, int32_t k_b, void* workspace,
                         size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
-/* cva_chunk_attention with the top-p block budget of cva_hsa_select_topp
+/* cva_chunk_attention (same passages: "Light Forcing" section 2.2 and the
+ * global time index of section 2B of the Causal-RoPE page) with the top-p
+ * block budget of cva_hsa_select_topp ("Sparse VideoGen2", section B)
  * (k_f >= 1, cap k_cap, threshold p in (0, 1]); workspace:
  * cva_chunk_workspace_bytes(shape, k_f, k_cap) bytes. */
 int cva_chunk_attention_topp(const void* q, const void* k, const void* v,
@@ -344,12 +358,16 @@ int cva_copy_rows_2d(const void* src, void* dst, int64_t n0, int64_t n1, int64_t
  * counterpart; this exists for callers that cannot allocate device memory
  * when they call, such as a plugin whose host runtime owns every allocation
  * and passes it only inputs and outputs, or a loop that forbids allocation
- * after start-up). Same arguments and results as cva_chunk_attention; the
- * scratch is one fixed 64 MiB array inside the library, held on every
- * device that loads it until the process exits. Shapes and budgets that
- * need more return CVA_ENOMEM without launching. Calls never allocate or
- * free memory. The first call on a device looks up the array's address
- * (cudaGetSymbolAddress), so make it before any stream capture. All calls
+ * after start-up). Same arguments, checks and results as cva_chunk_attention;
+ * the scratch is one fixed 64 MiB array inside the library (enough for the
+ * 1.3B-shaped 480P chunk at any budget up to 1024 candidate blocks). Shapes and
+ * budgets that need more return CVA_ENOMEM without launching. Under CUDA's
+ * default lazy module loading the array is reserved on a device by the first
+ * call there (which loads the library part that holds it and looks up its
+ * address with cudaGetSymbolAddress) and stays reserved until the process
+ * exits; that first call can fail for lack of device memory (CVA_ELAUNCH), so
+ * make it during start-up, before any stream capture, or set
+ * CUDA_MODULE_LOADING=EAGER. Later calls allocate and free nothing. All calls
  * share the one array and keep whatever the last call left in it: calls
  * that overlap on the GPU (different streams, or different host threads on
  * one device) race on it, so order them on one stream. */
@@ -372,6 +390,16 @@ int cva_set_stage_events(void* const* events, int32_t n);
  * x in [-125, 127]; inputs below -125 are clamped to it). Device buffers of
  * n floats. Not used by the path itself; it lets tests bound the error. */
 int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream);
+
+/* Diagnostic of the device-side failure path: one CTA waits, through the
+ * bounded wait every pipeline role of the kernels uses, on an mbarrier that
+ * nothing arrives at, with a limit of limit_us microseconds (1 .. 10^6)
+ * instead of the kernels' 4 s. The wait gives up, latches CVA_DEV_TIMEOUT in
+ * the device error word (read and cleared by cva_device_status) and raises
+ * the CTA's abort flag; result (device, 2 int32) receives {1 if the wait gave
+ * up, 1 if the abort flag was raised}. No copy or MMA is in flight, so the
+ * kernel returns normally and the context stays usable. */
+int cva_diag_wait_timeout(int32_t limit_us, int32_t* result, cva_stream_t stream);
 
 /* Chunk budget from the noise level ("Light Forcing", section 2.1: s_i =
  * s_base - alpha_i beta, alpha_i scaling with the noise level as 1/sqrt(T),

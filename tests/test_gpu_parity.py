@@ -19,7 +19,7 @@ from oracle import path as o_path
 from oracle import rope as o_rope
 
 from _util import (MAX_ABS, MEAN_ABS, attn_errors, bits_to_f64, f64_to_bits, from_dev, inputs,
-                   lib_budget, oracle_budget, hist_count, rope_tol, sample_rows, selection_mismatch,
+                   lib_budget, oracle_budget, hist_count, rope_tol, sample_rows, check_selection, ws_lists, oracle_run,
                    shape_of, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -46,34 +46,7 @@ def _sub(wl, heads):
     return wl if heads is None else wl.replace(H=len(heads))
 
 
-def _oracle_run(wl, chunk, heads=None, t_begin=0, topp=None, cap=None):
-    """Oracle over the window's chunks; returns per-chunk bf16 values and the
-    final chunk's path outputs (selection, pooled queries) without attention.
-    With ``topp`` the blocks follow the top-p budget with cap ``cap``."""
-    H = wl.H if heads is None else len(heads)
-    cache = o_path.FrameCache(wl.B, H, wl.D, wl.T_f, wl.blk, wl.window)
-    cache.t_begin = t_begin
-    centres = key_centres(wl, 0) if wl.keys == "clustered" else None
-    t0_cur = wl.t0_of(chunk) + t_begin
-    lo = max(t_begin, t0_cur + wl.Fc - wl.window)
-    first = (lo - t_begin) // wl.Fc + 1
-    hist = []
-    for c in range(first, chunk):
-        x = inputs(wl, c, 0, heads, centres)
-        q, k, v = (bits_to_f64(x[n]) for n in ("q", "k", "v"))
-        t0 = wl.t0_of(c) + t_begin
-        _, k_rot = o_path.rotate_chunk(q, k, wl.Fh, wl.Fw, wl.Fc, t0, "bf16")
-        cache.append(k_rot, v, t0, wl.Fc)
-        hist.append((t0, k_rot, x["v"]))
-    x = inputs(wl, chunk, 0, heads, centres)
-    q, k, v = (bits_to_f64(x[n]) for n in ("q", "k", "v"))
-    k_f, k_b = oracle_budget(wl, chunk, t_begin)
-    if topp is not None:
-        k_b = cap
-    out = o_path.run_chunk(cache, q, k, v, Fh=wl.Fh, Fw=wl.Fw, Fc=wl.Fc, t0=t0_cur, k_f=k_f, k_b=k_b,
-                           dense=wl.dense, store="bf16", attend_too=False, topp=topp)
-    out.update(cache=cache, hist=hist, x=x, t0=t0_cur, k_f=k_f, k_b=k_b)
-    return out
+_oracle_run = oracle_run
 
 
 def _head_major(wl, q_rot_tok):
@@ -242,7 +215,7 @@ def test_hsa_select_staged(ops, key):
     wl = WORKLOADS[key]
     run = _oracle_run(wl, wl.chunk)
     _, _, fi, bi, bc = _staged_select(ops, wl, run)
-    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    n, bad, near, _ = check_selection(run, fi, bi, bc)
     assert bad == 0 and near <= 0.02 * n, (bad, near, n)
     kfe = run["frames"].shape[-1]
     ok = (run["gap_f"] >= 1e-5)
@@ -257,7 +230,7 @@ def test_hsa_select_staged_c3_full_size(ops, chunk):
     k_f, k_b = lib_budget(wl, chunk)
     assert (k_f, k_b) == (run["k_f"], run["k_b"])
     _, _, fi, bi, bc = _staged_select(ops, _sub(wl, heads), run)
-    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    n, bad, near, _ = check_selection(run, fi, bi, bc)
     assert bad == 0 and near <= 0.02 * n, (bad, near, n)
 
 
@@ -275,7 +248,7 @@ def test_select_and_attention_at_the_size_limits(ops, k_b):
     assert run["k_f"] == 256 and run["k_b"] == k_b and len(run["hist"]) == 86
     assert run["frames"].shape[-1] == 256 and run["blocks"].shape[-1] == k_b
     _, _, fi, bi, bc = _staged_select(ops, wl, run)
-    n, bad, near = selection_mismatch(bi, bc, run["blocks"], run["gap_f"], run["gap_b"])
+    n, bad, near, _ = check_selection(run, fi, bi, bc)
     assert bad == 0 and near <= 0.1 * n, (bad, near, n)
     _check_attention(ops, wl, run, run["blocks"], split=True)
 
@@ -372,38 +345,28 @@ def _gpu_stream(ops, wl, upto, t_begin=0, heads=None, record=()):
     return res, cache
 
 
-def _e2e_compare(wl, run, gpu_out, blocks_ok=None, rows=None):
-    """Output of the fused call vs the oracle; query blocks where the
-    selection differed (near ties) are excluded."""
-    o_want, _ = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, run["blocks"], rows)
+def _e2e_compare(wl, run, gpu_out, blocks=None, rows=None):
+    """Output of the fused call vs the oracle over every compared row. ``blocks``
+    are the key sets to attend (default: the oracle's selection); where the
+    GPU's selection differed validly at a near-tie, :func:`_e2e_selection`
+    substitutes the GPU's own lists so that those rows are compared too."""
+    use = run["blocks"] if blocks is None else blocks
+    o_want, _ = o_path.attend_chunk(run["q_rot"], run["cache"], run["t0"], wl.Fc, use, rows)
     got = bits_to_f64(gpu_out)
     sel = np.arange(wl.Lq) if rows is None else rows
-    g = got[:, sel]
-    w = o_want[:, sel]
-    if blocks_ok is not None:
-        qb = (sel // wl.T_f) * wl.nb + (sel % wl.T_f) // wl.blk
-        mask = blocks_ok[:, :, qb]                          # [B, H, rows]
-        mask = np.transpose(mask, (0, 2, 1))[..., None]     # [B, rows, H, 1]
-        g = np.where(mask, g, 0.0)
-        w = np.where(mask, w, 0.0)
-    return attn_errors(g, w)
+    return attn_errors(got[:, sel], o_want[:, sel])
 
 
-def _selection_ok_mask(run, gpu_blocks):
-    if run["blocks"] is None:
-        return None
-    kb = run["blocks"].shape[-1]
-    return np.all(gpu_blocks[..., :kb] == run["blocks"], axis=-1)
-
-
-def _ws_blocks(ops, wl, ws, k_f, k_b):
-    """Block lists the fused call wrote into its workspace (layout of cva_chunk_workspace_bytes)."""
-    d = wl
-    bhq = d.B * d.H * d.NQB
-    r256 = lambda x: (x + 255) // 256 * 256
-    off = r256(d.B * d.H * d.Fc * d.T_pad * d.D * 2) + r256(bhq * d.D * 4) + r256(bhq * max(k_f, 0) * 4)
-    raw = ws[off:off + bhq * k_b * 4].cpu().numpy().view(np.int32)
-    return raw.reshape(d.B, d.H, d.NQB, k_b)
+def _e2e_selection(wl, run, ws, k_f, k_b, heads=None, max_near=0.02):
+    """Checks the fused call's selection against the oracle (:func:`check_selection`)
+    and returns the key sets its attention used."""
+    kfe = run["frames"].shape[-1]
+    fr, bl, ct = ws_lists(wl, ws, k_f, k_b, kfe)
+    if heads is not None:
+        fr, bl, ct = fr[:, heads], bl[:, heads], ct[:, heads]
+    n, bad, near, blocks = check_selection(run, fr, bl, ct)
+    assert bad == 0 and near <= max_near * n, (bad, near, n)
+    return blocks
 
 
 @pytest.mark.parametrize("key", SMALL)
@@ -412,12 +375,10 @@ def test_chunk_attention_end_to_end(ops, key):
     res, _ = _gpu_stream(ops, wl, wl.chunk)
     out, ws, k_f, k_b = res[wl.chunk]
     run = _oracle_run(wl, wl.chunk)
-    ok = None
+    blocks = None
     if not wl.dense and k_b > 0:
-        gb = _ws_blocks(ops, wl, ws, k_f, k_b)
-        ok = _selection_ok_mask(run, gb)
-        assert ok.mean() >= 0.98, ok.mean()
-    mx, mean, rel = _e2e_compare(wl, run, out, ok)
+        blocks = _e2e_selection(wl, run, ws, k_f, k_b)
+    mx, mean, rel = _e2e_compare(wl, run, out, blocks)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -441,9 +402,8 @@ def test_chunk_attention_rolling_window_wrap(ops):
     out, ws, k_f, k_b = res[7]
     run = _oracle_run(wl, 7)
     assert cache.history_frames(run["t0"]) == (13, 5)
-    gb = _ws_blocks(ops, wl, ws, k_f, k_b)
-    ok = _selection_ok_mask(run, gb)
-    mx, mean, _ = _e2e_compare(wl, run, out, ok)
+    blocks = _e2e_selection(wl, run, ws, k_f, k_b)
+    mx, mean, _ = _e2e_compare(wl, run, out, blocks)
     assert mx <= MAX_ABS and mean <= MEAN_ABS
 
 
@@ -473,11 +433,9 @@ def test_c3_hsa_end_to_end_sampled(ops, chunk):
     out, ws, k_f, k_b = res[chunk]
     heads = [1, 6]
     run = _oracle_run(wl, chunk, heads)
-    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
-    ok = _selection_ok_mask(run, gb)
-    assert ok.mean() >= 0.98, ok.mean()
+    blocks = _e2e_selection(wl, run, ws, k_f, k_b, heads)
     rows = sample_rows(wl, 1, np.random.default_rng(4))
-    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], blocks, rows)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -487,11 +445,9 @@ def test_c4_end_to_end_sampled(ops):
     res, _ = _gpu_stream(ops, wl, wl.chunk)
     out, ws, k_f, k_b = res[wl.chunk]
     run = _oracle_run(wl, wl.chunk, heads)
-    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
-    ok = _selection_ok_mask(run, gb)
-    assert ok.mean() >= 0.98, ok.mean()
+    blocks = _e2e_selection(wl, run, ws, k_f, k_b, heads)
     rows = sample_rows(wl, 1, np.random.default_rng(5), blocks=range(0, wl.NQB, 3))
-    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], blocks, rows)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -505,11 +461,9 @@ def test_c5_streaming_window_sampled(ops):
     assert (k_f, k_b) == (20, 285)
     assert cache.history_frames(wl.t0_of(21)) == (3, 57)
     run = _oracle_run(wl, 21, heads)
-    gb = _ws_blocks(ops, wl, ws, k_f, k_b)[:, heads]
-    ok = _selection_ok_mask(run, gb)
-    assert ok.mean() >= 0.98, ok.mean()
+    blocks = _e2e_selection(wl, run, ws, k_f, k_b, heads)
     rows = sample_rows(wl, 1, np.random.default_rng(6), blocks=range(0, wl.NQB, 4))
-    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], blocks, rows)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -526,8 +480,11 @@ def _topp_compare(wl, run, gpu_blocks, gpu_cnt, p, cap, tol=1e-4):
     """Per (b, h, query block): identical to the oracle, or, where it differs,
     still a valid top-p choice under the oracle's own ranking (a prefix of it
     whose cut lies within `tol` of p in share, or at a score near-tie).
-    Returns (units, mismatches that are not valid, valid mismatches)."""
+    Returns (units, mismatches that are not valid, valid mismatches, blocks):
+    ``blocks`` is the oracle's lists with every validly differing unit's list
+    replaced by the GPU's (padded with -1), the key sets the GPU attended."""
     B, H, NQB, _ = run["blocks"].shape
+    blocks = run["blocks"].copy()
     bad = near = 0
     for b in range(B):
         for h in range(H):
@@ -540,6 +497,8 @@ def _topp_compare(wl, run, gpu_blocks, gpu_cnt, p, cap, tol=1e-4):
                     continue
                 if run["gap_f"][b, h, qb] < 1e-5:         # the frames themselves were a near tie
                     near += 1
+                    blocks[b, h, qb] = -1
+                    blocks[b, h, qb, :r] = got
                     continue
                 ft = run["frames"][b, h, qb]
                 kb = np.stack([run["cache"].frames[t]["kb"][b, h] for t in ft])
@@ -554,9 +513,11 @@ def _topp_compare(wl, run, gpu_blocks, gpu_cnt, p, cap, tol=1e-4):
                     ok = False                               # stopped before reaching p
                 if ok:
                     near += 1
+                    blocks[b, h, qb] = -1
+                    blocks[b, h, qb, :r] = got
                 else:
                     bad += 1
-    return B * H * NQB, bad, near
+    return B * H * NQB, bad, near, blocks
 
 
 def _staged_select_topp(ops, wl, run, p, cap):
@@ -583,7 +544,7 @@ def test_hsa_select_topp_staged(ops, key, p):
     run = _oracle_run(wl, wl.chunk, topp=p, cap=cap)
     fi, bi, bc = _staged_select_topp(ops, wl, run, p, cap)
     assert np.all((bc >= 1) & (bc <= cap))
-    n, bad, near = _topp_compare(wl, run, bi, bc, p, cap)
+    n, bad, near, _ = _topp_compare(wl, run, bi, bc, p, cap)
     assert bad == 0 and near <= 0.05 * n, (bad, near, n)
     kfe = run["frames"].shape[-1]
     ok = run["gap_f"] >= 1e-5
@@ -596,7 +557,7 @@ def test_hsa_select_topp_cap_binds(ops):
     _, cap = _topp_cap(wl, wl.chunk, "budget")
     run = _oracle_run(wl, wl.chunk, topp=0.999, cap=cap)
     _, bi, bc = _staged_select_topp(ops, wl, run, 0.999, cap)
-    n, bad, near = _topp_compare(wl, run, bi, bc, 0.999, cap)
+    n, bad, near, _ = _topp_compare(wl, run, bi, bc, 0.999, cap)
     assert bad == 0 and near <= 0.05 * n, (bad, near, n)
     runk = _oracle_run(wl, wl.chunk)
     full = np.all(run["blocks"] >= 0, axis=-1)
@@ -611,7 +572,7 @@ def test_hsa_select_topp_c3_full_size(ops, chunk, p):
     _, cap = _topp_cap(wl, chunk, "all")
     run = _oracle_run(wl, chunk, heads, topp=p, cap=cap)
     fi, bi, bc = _staged_select_topp(ops, _sub(wl, heads), run, p, cap)
-    n, bad, near = _topp_compare(_sub(wl, heads), run, bi, bc, p, cap)
+    n, bad, near, _ = _topp_compare(_sub(wl, heads), run, bi, bc, p, cap)
     assert bad == 0 and near <= 0.05 * n, (bad, near, n)
 
 
@@ -636,12 +597,8 @@ def _gpu_stream_topp(ops, wl, upto, p, which):
         ops.chunk_attention_topp(*args, k_f, cap, p, ws, out)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
-    gb = _ws_blocks(ops, wl, ws, k_f, cap)
-    bhq = wl.B * wl.H * wl.NQB
-    r256 = lambda n: (n + 255) // 256 * 256
-    off = (r256(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D * 2) + r256(bhq * wl.D * 4) + r256(bhq * k_f * 4)
-           + r256(bhq * cap * 4))
-    gc = ws[off:off + bhq * 4].cpu().numpy().view(np.int32).reshape(wl.B, wl.H, wl.NQB)
+    kfe = min(k_f, hist_count(wl, upto))
+    _, gb, gc = ws_lists(wl, ws, k_f, cap, kfe)
     return from_dev(out), gb, gc, cap
 
 
@@ -650,10 +607,9 @@ def test_chunk_attention_topp_end_to_end(ops, key, p):
     wl = WORKLOADS[key]
     out, gb, gc, cap = _gpu_stream_topp(ops, wl, wl.chunk, p, "all")
     run = _oracle_run(wl, wl.chunk, topp=p, cap=cap)
-    n, bad, near = _topp_compare(wl, run, gb, gc, p, cap)
+    n, bad, near, blocks = _topp_compare(wl, run, gb, gc, p, cap)
     assert bad == 0 and near <= 0.05 * n, (bad, near, n)
-    ok = np.all(np.where(np.arange(cap) < gc[..., None], gb, -1) == run["blocks"], axis=-1)
-    mx, mean, rel = _e2e_compare(wl, run, out, ok)
+    mx, mean, rel = _e2e_compare(wl, run, out, blocks)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -664,11 +620,10 @@ def test_c3_topp_end_to_end_sampled(ops):
     heads = [1, 6]
     run = _oracle_run(wl, 7, heads, topp=p, cap=cap)
     gb, gc = gb[:, heads], gc[:, heads]
-    n, bad, near = _topp_compare(_sub(wl, heads), run, gb, gc, p, cap)
+    n, bad, near, blocks = _topp_compare(_sub(wl, heads), run, gb, gc, p, cap)
     assert bad == 0 and near <= 0.05 * n, (bad, near, n)
-    ok = np.all(np.where(np.arange(cap) < gc[..., None], gb, -1) == run["blocks"], axis=-1)
     rows = sample_rows(wl, 1, np.random.default_rng(7))
-    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], ok, rows)
+    mx, mean, rel = _e2e_compare(_sub(wl, heads), run, out[:, :, heads], blocks, rows)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
@@ -749,6 +704,25 @@ def test_bad_block_index_is_latched_not_read(ops):
     torch.cuda.synchronize()
     assert ops.device_status(clear=True) == ops.DEV_BAD_INDEX
     assert ops.device_status() == 0
+
+
+def test_bounded_wait_gives_up_and_latches_a_timeout(ops):
+    # one CTA waits on an mbarrier nothing arrives at, with a 2 ms limit: the
+    # wait returns, the timeout is latched and read back, the word clears, and
+    # the context is still usable (a normal launch afterwards runs)
+    import torch
+    res = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    assert ops.device_status(clear=True) == 0
+    ops.diag_wait_timeout(2000, res)
+    torch.cuda.synchronize()
+    assert res.cpu().tolist() == [1, 1]
+    assert ops.device_status(clear=True) == ops.DEV_TIMEOUT
+    assert ops.device_status() == 0
+    with pytest.raises(ops.CvaError) as e:
+        ops.diag_wait_timeout(0, res)
+    assert e.value.code == ops.CVA_EINVAL
+    y = torch.arange(8, dtype=torch.float32, device="cuda") + 1
+    assert float(y.sum()) == 36.0
 
 
 def test_host_errors(ops):

@@ -577,3 +577,83 @@ def test_denoising_passes_leave_no_trace():
     a, b = run(0), run(2)
     for c in (2, 3, 4):
         np.testing.assert_array_equal(a[c]["o"], b[c]["o"])
+
+
+# --- attention on ragged frames (several blocks per frame, a short tail) -----------
+#
+# Frames of 5 x 9 = 45 tokens over 16-token blocks: blocks [0, 16), [16, 32) and
+# the 13-token tail [32, 45). Two history frames (t = 0, 1) and a chunk of two
+# frames (t = 2, 3) whose 90 queries form six query blocks. The rows of each
+# query block and the token range of each picked block are written out by hand
+# below (not derived from the block size), so a slip in the oracle's row -> query
+# block map or in its tail slicing changes some key set and fails the test.
+
+_RAG_D, _RAG_TF, _RAG_BLK = 16, 45, 16
+# query block -> rows of the chunk (frame 2 holds rows 0..44, frame 3 rows 45..89)
+_RAG_QROWS = {0: range(0, 16), 1: range(16, 32), 2: range(32, 45),
+              3: range(45, 61), 4: range(61, 77), 5: range(77, 90)}
+# block id t*3 + j -> (frame t, first token, end token) of the picked history block
+_RAG_BLOCKS = {0: (0, 0, 16), 1: (0, 16, 32), 2: (0, 32, 45),
+               3: (1, 0, 16), 4: (1, 16, 32), 5: (1, 32, 45)}
+# picks per query block (ascending ids, as the selection reports them)
+_RAG_PICKS = {0: [2], 1: [1, 3], 2: [2, 5], 3: [0, 4], 4: [3, 4, 5], 5: [1]}
+
+
+def _ragged_case():
+    rng = np.random.default_rng(4242)
+    D, T_f = _RAG_D, _RAG_TF
+    hist_k = rng.standard_normal((1, 2 * T_f, 1, D))
+    hist_v = rng.standard_normal((1, 2 * T_f, 1, D))
+    cur_k = rng.standard_normal((1, 2 * T_f, 1, D))
+    cur_v = rng.standard_normal((1, 2 * T_f, 1, D))
+    q = rng.standard_normal((1, 2 * T_f, 1, D))
+    cache = path.FrameCache(1, 1, D, T_f, _RAG_BLK, window=8)
+    cache.append(hist_k, hist_v, 0, 2)
+    cache.append(cur_k, cur_v, 2, 2)
+    blocks = np.zeros((1, 1, 6, 3), dtype=np.int64) - 1
+    for qb, ids in _RAG_PICKS.items():
+        blocks[0, 0, qb, :len(ids)] = ids
+    return cache, q, blocks, (hist_k, hist_v, cur_k, cur_v)
+
+
+def _ragged_keys_by_hand(qb, raw):
+    hist_k, hist_v, cur_k, cur_v = raw
+    ks, vs = [], []
+    for g in _RAG_PICKS[qb]:
+        t, lo, hi = _RAG_BLOCKS[g]
+        ks.append(hist_k[0, t * _RAG_TF + lo:t * _RAG_TF + hi, 0])
+        vs.append(hist_v[0, t * _RAG_TF + lo:t * _RAG_TF + hi, 0])
+    ks.append(cur_k[0, :, 0])                  # the whole current chunk
+    vs.append(cur_v[0, :, 0])
+    return np.concatenate(ks), np.concatenate(vs)
+
+
+def test_ragged_frames_key_sets_match_hand_built_ranges():
+    cache, q, blocks, raw = _ragged_case()
+    for qb in range(6):
+        k, v = path.keys_of_query_block(cache, 0, 0, 2, 2, blocks[0, 0, qb])
+        kw, vw = _ragged_keys_by_hand(qb, raw)
+        np.testing.assert_array_equal(k, kw)
+        np.testing.assert_array_equal(v, vw)
+    # the tail blocks hold 13 tokens, the others 16
+    k2, _ = path.keys_of_query_block(cache, 0, 0, 2, 2, np.array([2]))
+    assert k2.shape[0] == 13 + 90
+
+
+def test_ragged_frames_attention_brute_force():
+    cache, q, blocks, raw = _ragged_case()
+    o, lse = path.attend_chunk(q, cache, 2, 2, blocks)
+    scale = 1 / math.sqrt(_RAG_D)
+    seen = set()
+    for qb, rows in _RAG_QROWS.items():
+        K, V = _ragged_keys_by_hand(qb, raw)
+        for r in rows:
+            s = scale * K @ q[0, r, 0]
+            np.testing.assert_allclose(o[0, r, 0], scipy.special.softmax(s) @ V, rtol=1e-11, atol=1e-13)
+            np.testing.assert_allclose(lse[0, 0, r], scipy.special.logsumexp(s), rtol=1e-13)
+            seen.add(r)
+    assert seen == set(range(90))
+    # a row subset gives the same numbers for those rows
+    rows = np.array([0, 31, 32, 44, 45, 60, 61, 89])
+    o2, _ = path.attend_chunk(q, cache, 2, 2, blocks, rows)
+    np.testing.assert_allclose(o2[0, rows], o[0, rows], rtol=1e-13, atol=1e-15)
