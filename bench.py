@@ -10,12 +10,19 @@ another buffer so that no dirty line of the flush is left to be written
 back inside the timed step) and only the step itself is timed (CUDA events
 on the launching stream).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4]
     python bench.py --impl reference      # the fp64 oracle on the host cores
 
-Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its
-own independent instance (its own seeded layer): weak scaling, no data-path
-collective; the reported time is the max over ranks.
+Prints one JSON line (rank 0). The line's workload is c4 (the 14B-shaped
+720P chunk with hierarchical selection, the largest single-GPU
+configuration); on one GPU the line also carries ``per_config`` entries
+measured in the same run: c2 (1.3B-shaped dense chunk), c3 chunk 7 (1.3B
+shape, hierarchical selection) and c5 (80 chunks x 30 layers streamed
+through a rolling window, per-chunk latency p50/p99). With N > 1
+(torchrun) every rank runs its own independent instance of the line's
+workload (its own seeded layer): weak scaling, no data-path collective; the
+reported time is the max over ranks, and the per-config entries are left
+out.
 """
 from __future__ import annotations
 
@@ -43,12 +50,14 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--workload", default="c2")
+    ap.add_argument("--workload", default="c4")
     ap.add_argument("--chunk", type=int, default=None, help="chunk index (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config entries (c2 dense, c3 chunk 7, c5 streaming) of the line")
     ap.add_argument("--sweep", action="store_true",
                     help="chunks 1..N of the workload under its literal and mirrored density "
                          "schedules, one JSON line each (measurement mode, not the bench line)")
@@ -422,6 +431,88 @@ def config_of(wl):
             "t0": wl.t0, "budget": "dense" if wl.dense else "hierarchical sparse"}
 
 
+def measure_chunk(args, wl, layer, stream, flush, n, clocks_on, world=1):
+    """Times one chunk of `wl` through the fused call: warm-up, then n steps
+    with L2 flushed before each, clocks sampled during the timed steps.
+    Returns the device state and the per-step stage times (ms)."""
+    import torch
+    import torch.distributed as dist
+    from autoregressive_video_dit_b200 import ops
+
+    st = setup_workload(args, layer=layer, wl=wl)
+    wl = st["wl"]
+
+    def step():
+        ops.chunk_attention(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0, st["k_f"],
+                            st["k_b"], st["ws"], st["out"])
+
+    for _ in range(max(args.warmup, 1)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    flops = attention_flops(st)
+    sampler = ClockSampler(enabled=clocks_on)
+    time.sleep(0.3 if clocks_on else 0)
+    if world > 1:
+        dist.barrier()
+    step_ms, rope_ms, sel_ms, attn_ms = time_steps(step, flush, n, stream)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    assert ops.device_status() == 0
+    return dict(st=st, step=step, flops=flops, step_ms=step_ms, rope_ms=rope_ms, sel_ms=sel_ms,
+                attn_ms=attn_ms, clocks=clocks)
+
+
+def attention_peak(peaks, clocks):
+    """The burst bf16 figure for a kernel that ran at full clock; the
+    sustained one when the timed region ran into the power cap (a long step)."""
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    peak = float(peaks["bf16_tflops_sustained" if capped else "bf16_tflops"])
+    kind = "bf16 sustained (power cap seen while timing)" if capped else "bf16 burst"
+    return peak, kind
+
+
+def config_entry(m, peaks, peak_src):
+    """Per-config summary of one measure_chunk() result."""
+    st, wl = m["st"], m["st"]["wl"]
+    ms = statistics.mean(m["step_ms"])
+    attn = statistics.mean(m["attn_ms"])
+    rope = statistics.mean(m["rope_ms"])
+    sel = statistics.mean(m["sel_ms"])
+    peak, kind = attention_peak(peaks, m["clocks"])
+    ach = m["flops"] / (attn * 1e-3) / 1e12
+    rb = rope_bytes(wl)
+    return {
+        "workload": f"{wl.key}: {wl.name}", "chunk_index": wl.chunk, "history_frames": st["F"],
+        "k_f": st["k_f"], "k_b": st["k_b"], "budget": "dense" if wl.dense else "hierarchical sparse",
+        "ms": ms, "attention_tflop": m["flops"] / 1e12,
+        "effective_tflops": m["flops"] / (ms * 1e-3) / 1e12,
+        "attention_ms": attn, "attention_tflops": ach,
+        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": ach, "peak": peak,
+                     "unit": "TFLOP/s", "frac": ach / peak,
+                     "peak_source": f"{peak_src} {kind}", "flops": "useful: each query block's own keys"},
+        "rotate_append_pool_us": 1e3 * rope,
+        "roofline_hbm": {"kernel": "rope_pool_tma_kernel", "bound": "hbm",
+                         "achieved": rb / (rope * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
+                         "unit": "GB/s", "frac": rb / (rope * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                         "algorithmic_bytes": rb},
+        "select_us": 1e3 * sel, "select_share": sel / ms,
+        "steps": len(m["step_ms"]), "stat": "mean", "clocks": m["clocks"],
+    }
+
+
+def stream_entry(args, clocks_on, chunks=None):
+    """c5 streaming: every chunk through all layers (run_stream's loop),
+    per-chunk latency p50/p99 with clocks sampled over the run."""
+    sampler = ClockSampler(enabled=clocks_on)
+    res = stream_latencies(args, "c5", chunks)
+    clocks = sampler.stop()
+    res["clocks"] = clocks
+    return res
+
+
 def run_cuda(args):
     import torch
     import torch.distributed as dist
@@ -434,35 +525,19 @@ def run_cuda(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     from autoregressive_video_dit_b200 import ops
+    from cva_workload import WORKLOADS
 
-    st = setup_workload(args, layer=rank_layer(rank))
-    wl = st["wl"]
+    wl = WORKLOADS[args.workload]
+    if args.chunk is not None:
+        wl = wl.with_chunk(args.chunk)
     stream = torch.cuda.current_stream()
     flush = L2Flush()
-
-    def step():
-        ops.chunk_attention(st["q"], st["k"], st["v"], st["cache"], st["tables"], wl.t0, st["k_f"],
-                            st["k_b"], st["ws"], st["out"])
-
-    for _ in range(max(args.warmup, 1)):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    assert ops.device_status() == 0
-    flops = attention_flops(st)
-
     n = args.steps
-    sampler = ClockSampler(enabled=not args.no_clocks)
-    time.sleep(0.3 if not args.no_clocks else 0)
-    if world > 1:
-        dist.barrier()
-    step_ms, rope_ms, sel_ms, attn_ms = time_steps(step, flush, n, stream)
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    assert ops.device_status() == 0
+    m = measure_chunk(args, wl, rank_layer(rank), stream, flush, n, not args.no_clocks, world)
+    st, step, flops, clocks = m["st"], m["step"], m["flops"], m["clocks"]
+    wl = st["wl"]
 
-    ms = statistics.mean(step_ms)
+    ms = statistics.mean(m["step_ms"])
     ms_max, total_flops = reduce_over_ranks(ms, flops, "cuda")
 
     # end to end through the public call with pinned host buffers
@@ -498,16 +573,8 @@ def run_cuda(args):
         return 0
 
     peaks, peak_src = load_peaks()
-    attn_avg = statistics.mean(attn_ms)
-    achieved = flops / (attn_avg * 1e-3) / 1e12
-    # the burst figure for a kernel that ran at full clock; the sustained one
-    # when the timed region ran into the power cap (a long step)
-    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
-    peak = float(peaks["bf16_tflops_sustained" if capped else "bf16_tflops"])
-    peak_kind = "bf16 sustained (power cap seen while timing)" if capped else "bf16 burst"
+    entry = config_entry(m, peaks, peak_src)
     traffic = recorded_traffic("attn_sm100.cu", wl.key)
-    rope_avg = statistics.mean(rope_ms)
-    rb = rope_bytes(wl)
     line = {
         "metric": METRIC,
         "value": total_flops / (ms_max * 1e-3) / 1e12,
@@ -526,24 +593,28 @@ def run_cuda(args):
                        parallelism="independent instance per GPU" if world > 1 else "1 GPU"),
         "latency_ms": ms_max,
         "attention_tflop_per_chunk": flops / 1e12,
-        "frac_of_bf16_peak": (total_flops / world) / (ms_max * 1e-3) / 1e12 / peak,
-        "stage_ms": {"rotate_append_pool": rope_avg, "select": statistics.mean(sel_ms),
-                     "attention": attn_avg},
-        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": traffic, "peak_source": f"{peak_src} {peak_kind}"},
-        "roofline_hbm": {"kernel": "rope_pool_kernel", "bound": "hbm",
-                         "achieved": rb / (rope_avg * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
-                         "unit": "GB/s", "frac": rb / (rope_avg * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
-                         "algorithmic_bytes": rb},
-        # rotate/append/pool; selection and (64-row blocks, history of at least 2 k_f frames)
-        # query-block pairing; attention (+ merge)
-        "gpu_launches": n * (1 + ((1 + (wl.blk == 64 and st["F"] >= 2 * min(st["k_f"], st["F"])))
-                                  if (st["k_f"] >= 0 and st["F"] > 0) else 0) + attention_launches(wl)),
+        "frac_of_bf16_peak": (total_flops / world) / (ms_max * 1e-3) / 1e12 / entry["roofline"]["peak"],
+        "stage_ms": {"rotate_append_pool": entry["rotate_append_pool_us"] * 1e-3,
+                     "select": entry["select_us"] * 1e-3, "attention": entry["attention_ms"]},
+        "roofline": dict(entry["roofline"], traffic=traffic),
+        "roofline_hbm": entry["roofline_hbm"],
+        "gpu_launches": n * launches_per_step(wl, st),
         "clocks": clocks,
     }
     if e2e:
         line["e2e"] = e2e
+    if world == 1 and not args.no_per_config:
+        per = {}
+        for key, chunk in (("c2", None), ("c3", 7)):
+            if key == wl.key and (chunk is None or chunk == wl.chunk):
+                continue
+            w2 = WORKLOADS[key] if chunk is None else WORKLOADS[key].with_chunk(chunk)
+            m2 = measure_chunk(args, w2, 0, stream, flush, n, not args.no_clocks)
+            per[key] = config_entry(m2, peaks, peak_src)
+            del m2
+            torch.cuda.empty_cache()
+        per["c5"] = stream_entry(args, not args.no_clocks)
+        line["per_config"] = per
     if world == 1 and not args.no_cpu_baseline:
         n_aff, threads = host_cores()
         v, desc, dt, _ = OracleSample(wl).run(args.cpu_seconds)
@@ -554,6 +625,18 @@ def run_cuda(args):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def launches_per_step(wl, st):
+    """Kernel launches of one fused chunk call: rotate/append/pool; the
+    selection (sparse budget with history) and the query-block pairing (64-row
+    blocks, a history of at least 2 k_f frames); the attention, plus the merge
+    of split tail tiles."""
+    sparse = st["k_f"] >= 0 and st["F"] > 0
+    n = 1 + attention_launches(wl)
+    if sparse:
+        n += 1 + int(wl.blk == 64 and st["F"] >= 2 * min(st["k_f"], st["F"]))
+    return n
 
 
 def run_sweep(args):
@@ -618,16 +701,17 @@ def run_sweep(args):
     return 0
 
 
-def run_stream(args):
-    """Every chunk of the workload once, through all its layers, each layer
-    with its own cache (rolling window); per-chunk latency = the sum over
-    layers, timed from the first layer's start to the last layer's end.
-    Inputs are drawn on the device from a seeded generator per (chunk,
-    layer), outside the timed region."""
+def stream_latencies(args, key, chunks=None):
+    """Every chunk of the workload once (or the first `chunks`), through all
+    its layers, each layer with its own cache (rolling window); per-chunk
+    latency = the sum over layers, timed from the first layer's start to the
+    last layer's end. Inputs are drawn on the device from a seeded generator
+    per (chunk, layer), outside the timed region."""
     import torch
     from autoregressive_video_dit_b200 import ops
     from cva_workload import WORKLOADS
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS[key]
+    nch = wl.chunks if chunks is None else chunks
     shape = ops.make_shape(wl.B, wl.H, wl.D, wl.Fh, wl.Fw, wl.Fc, wl.blk)
     tables = ops.DeviceRopeTables(wl.D, wl.Fc * wl.chunks, wl.Fh, wl.Fw)
     caches = [ops.DeviceKVCache(shape, wl.window, 0) for _ in range(wl.layers)]
@@ -666,17 +750,25 @@ def run_stream(args):
     for c in (1, 2):                      # warm-up, then the caches start over
         run_chunk(c, False)
     caches = [ops.DeviceKVCache(shape, wl.window, 0, arena=x.arena) for x in caches]
-    lat = [run_chunk(c, True) for c in range(1, wl.chunks + 1)]
+    lat = [run_chunk(c, True) for c in range(1, nch + 1)]
     assert ops.device_status() == 0
     full = wl.window // wl.Fc + 1          # first chunk whose history fills the window
     steady = lat[full - 1:]
-    print(json.dumps({
-        "mode": "streaming", "workload": wl.key, "chunks": wl.chunks, "layers": wl.layers,
+    res = {
+        "mode": "streaming", "workload": f"{wl.key}: {wl.name}", "chunks": nch, "layers": wl.layers,
         "window_frames": wl.window, "unit": "ms per chunk (all layers)",
         "p50": percentile(lat, 50), "p99": percentile(lat, 99), "max": max(lat),
-        "chunk1": lat[0], "steady_p50": percentile(steady, 50), "steady_from_chunk": full,
+        "chunk1": lat[0], "steady_p50": percentile(steady, 50) if steady else None,
+        "steady_from_chunk": full,
         "budget_first_full_window": {"k_f": budgets[full - 1][0], "k_b": budgets[full - 1][1]},
-        "per_chunk": [round(x, 3) for x in lat]}), flush=True)
+        "per_chunk": [round(x, 3) for x in lat]}
+    del caches, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_stream(args):
+    print(json.dumps(stream_latencies(args, args.workload)), flush=True)
     return 0
 
 
