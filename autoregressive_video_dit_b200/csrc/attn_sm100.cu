@@ -11,29 +11,40 @@
 // unit's mask says which of them picked it); an odd count is padded with an
 // empty unit.
 //
-// Tensor memory holds two score buffers S0 and S1 (128 fp32 columns each,
-// P aliased onto the scores it came from) and two output accumulators
-// O_even and O_odd (128 columns each). Key tile i's scores go to buffer
-// i mod 2 and its PV into O of the same parity. With two score buffers the
-// tensor core computes S(i+1) while the softmax works on S(i), and PV(i) is
-// followed right away by S(i+2) into the buffer P(i) leaves.
+// Tensor memory holds one output accumulator O (columns 0 .. D-1) and three
+// score buffers S0, S1, S2 (128 fp32 columns each at 128, 256, 384; P is
+// written back over the first 64 columns of its own scores). Key tile i goes
+// to buffer i mod 3, so the scores of the next two tiles are computed while
+// the softmax works on tile i: the chain S(i) -> softmax(i) -> PV(i) ->
+// S(i+3) has three links in flight and the tensor core does not wait for
+// one softmax to finish before the next tile's scores.
+//
+// The softmax of all tiles shares one running maximum per query row, so that
+// every PV accumulates into the one O: the online softmax keeps a reference
+// maximum m that only moves up, and only when a tile's row maximum exceeds it
+// by more than 2^8 (in the exponent); P = 2^(s/sqrt(D) log2 e - m) <= 2^8
+// otherwise. Tile i's warp needs m after tile i-1 before it can fix P(i): the
+// two warps of a row range hand m over through shared memory and an mbarrier
+// per direction, once per tile, right after their row maxima (early in the
+// tile). When m moves up at tile i the warp rescales its rows of O, after
+// PV(i-1) completed and before it releases P(i) (so before PV(i) is issued).
 //
 // Roles (384 threads):
 //   warps 0-3 / 4-7: softmax of the even / odd key tiles. Warps w and w + 4
-//     own query rows 32 (w mod 4) .. + 31 (TMEM lanes; thread = row); each
-//     runs its own online softmax over its tiles (all 128 key columns) into
-//     its own O, so the two warps sharing a scheduler work on different tiles
-//     and never wait for each other. Masks, row maximum (3-input max), exp2
-//     on the MUFU in fp32 with packed f32x2 arithmetic, bf16 P written back
-//     over the S columns. O is rescaled in tensor memory only when the row
-//     maximum grows by more than 2^8 (S(i) completing implies PV(i-2) did).
-//     At the end the pair merges its two (O, max, sum) and writes bf16 O.
+//     own query rows 32 (w mod 4) .. + 31 (TMEM lanes; thread = row). Masks,
+//     row maximum (3-input max), the hand-over of m, exp2 on the MUFU in fp32
+//     with packed f32x2 arithmetic, bf16 P written back over the S columns.
+//     Each warp keeps its own row sum relative to the m it last saw; at the
+//     end the pair merges the two sums and writes bf16 O (each warp half of
+//     the columns).
 //   warp 8 (one lane): TMA producer. Q once, then K and V of every tile in
-//     order into the ring slot t mod 2, each as soon as its slot is free,
-//     gathered by block index with one 64-row box per unit and 64-column
-//     chunk, 128-byte swizzle. No multicast.
+//     the order the MMAs consume them, K into ring slot t mod 2 and V into
+//     slot t mod 3, each as soon as its slot is free, gathered by block index
+//     with one 64-row box per unit and 64-column chunk, 128-byte swizzle. No
+//     multicast.
 //   warp 9 (one lane): tcgen05.mma issuer, in the fixed order S(0), S(1),
-//     PV(0), S(2), PV(1), S(3), ...
+//     S(2), PV(0), S(3), PV(1), S(4), ...
+//   warps 10-11: frame means of the chunk's new cache frames (fused call).
 // Every wait is bounded: on timeout the CTA latches CVA_DEV_TIMEOUT, all
 // roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait and the tensor memory is released.
@@ -46,21 +57,34 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace cva {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kStages = 2;
+constexpr int kKStages = 2;   // K ring slots (tile t in slot t mod 2)
+constexpr int kVStages = 3;   // V ring slots (tile t in slot t mod 3)
+constexpr int kSBufs = 3;     // score buffers in tensor memory
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-// 12 warps: registers are granted per group of four warps, so warps 10 and
-// 11 cost nothing extra; they only join the final barrier.
+// 12 warps in three warpgroups: the two softmax warpgroups, then the
+// producer, the MMA issuer and two warps for the frame means. The launch
+// grants 168 registers a thread (three warps per scheduler); after the key
+// stream is built the third warpgroup gives registers back (setmaxnreg.dec
+// to kRegsOther) and the softmax warpgroups take them (setmaxnreg.inc to
+// kRegsSoftmax): 2 * 128 * 224 + 128 * 56 = 384 * 168, exactly the launch's
+// registers, so the increase always completes.
 constexpr int kAttnThreads = 384;
-constexpr uint32_t kTmemCols = 512;   // S0 at 0, S1 at 128, O_even at 256, O_odd at 384
-constexpr uint32_t kOCol = 256;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsOther = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kAttnThreads * 168, "register split");
+constexpr uint32_t kTmemCols = 512;   // O at 0, S0 at 128, S1 at 256, S2 at 384
+constexpr uint32_t kOCol = 0;
+constexpr uint32_t kSCol = 128;
 
 template <int D>
 struct AttnSmem {
@@ -69,31 +93,46 @@ struct AttnSmem {
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // a Q, K or V tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;                // slot s at + s * tile
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kEnt = kV + kStages * kTileBytes;
-  // softmax epilogue exchange: (max, sum) [2 parities][128 rows], flags [2][4]
+  static constexpr int kV = kK + kKStages * kTileBytes;
+  static constexpr int kEnt = kV + kVStages * kTileBytes;
+  // softmax epilogue exchange: (max, sum) [2 parities][128 rows], flags [2][4];
+  // then the hand-over of the running maximum: [128 rows] floats
   static constexpr int kRed = kEnt + kAttnMaxEntries * 4;
-  static constexpr int kBar = kRed + 2 * 128 * 8 + 2 * 4 * 4;
+  static constexpr int kHand = kRed + 2 * 128 * 8 + 2 * 4 * 4;
+  static constexpr int kBar = kHand + 128 * 4;
   static constexpr int kMisc = kBar + 32 * 8;
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
   // While the key list is built, its bitmaps and counts live in the V ring.
   static constexpr int kBm = kV;                                   // 4 bitmaps
   static constexpr int kCnt = kBm + 4 * kAttnMaxBitmapWords * 4;   // 3 count arrays
-  static_assert(7 * kAttnMaxBitmapWords * 4 <= kStages * kTileBytes, "build scratch");
+  static_assert(7 * kAttnMaxBitmapWords * 4 <= kVStages * kTileBytes, "build scratch");
+  static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
-// Barriers: S buffer b full / P written into it; K and V ring slots full and
-// free; PV done (every PV), O final; one for draining the tensor pipe.
-constexpr int kBarSFull = 0, kBarPFull = 2, kBarKFull = 4, kBarKEmpty = 6, kBarVFull = 8,
-              kBarVEmpty = 10, kBarQ = 12, kBarODone = 13, kBarDrain = 14;
+// Barriers: S buffer b full / P written into it (3 each; S(j) completing also
+// frees K slot j mod 2); K ring slots full (2); V ring slots full and free
+// (3 each; V slot t mod 3
+// frees when PV(t) completes, so it also tells that PV(t) is done); Q; O
+// final; one for draining the tensor pipe; the hand-over of the running
+// maximum per row range: [quarter][0] even -> odd tiles, [quarter][1] odd ->
+// even tiles.
+constexpr int kBarSFull = 0, kBarPFull = 3, kBarKFull = 6, kBarVFull = 8, kBarVEmpty = 11,
+              kBarQ = 14, kBarODone = 15, kBarDrain = 16, kBarHand = 17;  // .. 24
+
+// Whether full tiles compute a share of their exponentials with the
+// polynomial exp2 (see poly_pair in cva_internal.cuh for the share). Off:
+// measured on the 1.3B-shaped dense chunk, every share (1/4 .. 1/2 of the
+// pairs) was slower than the MUFU alone (0.789 ms vs 0.824-0.879 ms).
+#ifndef CVA_ATTN_POLY
+#define CVA_ATTN_POLY 0
+#endif
+constexpr bool kAttnPoly = CVA_ATTN_POLY != 0;
 
 // Above this growth of the row maximum (log2 units) O is rescaled; below
 // it the stale maximum is kept, so P <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
 
-// Longest sleep of the idle producer on one barrier (ns).
-constexpr uint32_t kSleepNs = 1000;
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -261,7 +300,7 @@ __device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, ui
                               (((b3 >> bit) & 1u) << 3);
         const int vb = (j == d.nb - 1) ? d.tail : d.blk;
         for (int u = 0; u < upb; ++u) {
-          const int i = pos[cls]++;
+          const int i = cls == 0 ? pos[0]++ : (cls == 1 ? pos[1]++ : pos[2]++);
           const int e = cls == 0 ? i : st.private_entry(cls - 1, i);
           ents[e] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
         }
@@ -284,27 +323,30 @@ __device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, ui
   return st;
 }
 
+// The MMAs of one key tile, from shared-memory descriptors computed once per
+// CTA: the descriptor's start address field is the byte address / 16 in its
+// low 14 bits, and every operand lies below 256 KB, so the k-th step's
+// descriptor is the base plus a compile-time constant. (One thread issues
+// all MMAs; keeping its instruction stream short and free of dependent
+// chains is what lets it keep up with the tensor core.)
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t s_tmem, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_s(uint32_t s_tmem, uint64_t q_desc, uint64_t k_desc) {
   constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
-    const uint32_t off = (uint32_t)((k >> 2) * AttnSmem<D>::kChunkBytes + (k & 3) * 32);
-    mma_ss(s_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-           kIdS, k > 0 ? 1u : 0u);
+    const uint64_t off = (uint64_t)(((k >> 2) * AttnSmem<D>::kChunkBytes + (k & 3) * 32) >> 4);
+    mma_ss(s_tmem, q_desc + off, k_desc + off, kIdS, k > 0 ? 1u : 0u);
   }
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
                                          bool accumulate) {
   constexpr uint32_t kIdO = idesc_bf16_f32(kBM, D, 0, 1);    // P (tmem), V MN-major
 #pragma unroll
-  for (int k = 0; k < kBN / 16; ++k) {
-    mma_ts(o_tmem, p_tmem + (uint32_t)(k * 8),
-           smem_desc_sw128(v_addr + (uint32_t)(k * 2048), AttnSmem<D>::kChunkBytes, 1024), kIdO,
+  for (int k = 0; k < kBN / 16; ++k)
+    mma_ts(o_tmem, p_tmem + (uint32_t)(k * 8), v_desc + (uint64_t)((k * 2048) >> 4), kIdO,
            (accumulate || k > 0) ? 1u : 0u);
-  }
 }
 
 
@@ -336,14 +378,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&bar[kBarSFull + s], 1);
-      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps / 2);  // one warp set per buffer
+      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps / 2);  // one warp set per tile
+    }
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bar[kBarKFull + s], 1);
-      mbar_init(&bar[kBarKEmpty + s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bar[kBarVFull + s], 1);
       mbar_init(&bar[kBarVEmpty + s], 1);
     }
+    for (int h = 0; h < 8; ++h) mbar_init(&bar[kBarHand + h], 32);  // one warp's rows
     mbar_init(&bar[kBarQ], 1);
     mbar_init(&bar[kBarODone], 1);
     mbar_init(&bar[kBarDrain], 1);
@@ -367,131 +413,186 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      auto load_kv = [&](int t, bool is_v) {
-        const uint32_t e0 = units[2 * t], e1 = units[2 * t + 1];
-        const int r0 = (int)(e0 >> 16) * 64;
-        const int r1 = (int)(e1 >> 16) * 64;
-        const int s = t & 1;
-        uint64_t* full = &bar[(is_v ? kBarVFull : kBarKFull) + s];
-        uint8_t* dst = smem + (is_v ? L::kV : L::kK) + s * L::kTileBytes;
-        const CUtensorMap* map = is_v ? &tmV : &tmK;
-        mbar_arrive_expect_tx(full, L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(dst + c * L::kChunkBytes, map, full, c * 64, r0, bh);
-          tma_load_3d(dst + c * L::kChunkBytes + 8192, map, full, c * 64, r1, bh);
+  // Every role ends at this barrier (all 384 threads) before the tensor
+  // memory is released.
+  auto end_barrier = [] {
+    __syncwarp();
+    tc_fence_before();
+    asm volatile("bar.sync 15, %0;" ::"n"(kAttnThreads) : "memory");
+  };
+  if (warp >= kSoftmaxWarps) {
+    // warpgroup 2: producer, MMA issuer, frame means (few registers)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsOther));
+    if (warp == kProducerWarp) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        auto load_kv = [&](int t, bool is_v) {
+          const uint32_t e0 = units[2 * t], e1 = units[2 * t + 1];
+          const int r0 = (int)(e0 >> 16) * 64;
+          const int r1 = (int)(e1 >> 16) * 64;
+          const int s = is_v ? (t % kVStages) : (t % kKStages);
+          uint64_t* full = &bar[(is_v ? kBarVFull : kBarKFull) + s];
+          uint8_t* dst = smem + (is_v ? L::kV : L::kK) + s * L::kTileBytes;
+          const CUtensorMap* map = is_v ? &tmV : &tmK;
+          mbar_arrive_expect_tx(full, L::kTileBytes);
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_load_3d(dst + c * L::kChunkBytes, map, full, c * 64, r0, bh);
+            tma_load_3d(dst + c * L::kChunkBytes + 8192, map, full, c * 64, r1, bh);
+          }
+        };
+        if (N > 0) {
+          // the tile's two 64-row halves (a half with no query block reads past
+          // the chunk's rows: zero fill)
+          const int q0 = tile_row(a, bh, m, 0), q1 = tile_row(a, bh, m, 64);
+          const int past = a.d.Fc * a.d.T_pad;
+          mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, q0 < 0 ? past : q0, bh);
+            tma_load_3d(smem + L::kQ + c * L::kChunkBytes + 8192, &tmQ, &bar[kBarQ], c * 64, q1 < 0 ? past : q1, bh);
+          }
         }
+        // Loads in the order the MMAs consume them: K(0), K(1), K(2), then
+        // V(i), K(i + 3) for i = 0, 1, ... (PV(i) is followed by S(i + 3)). K(t)
+        // goes to slot t mod 2 once S(t - 2) completed (SFull of its buffer),
+        // V(t) to slot t mod 3 once PV(t - 3) completed. Each wait is for
+        // exactly the barrier the next load needs, so the producer wakes when
+        // that slot frees.
+        int kt = 0, vt = 0;
+        bool ok = true;
+        while (ok && (kt < N || vt < N)) {
+          if (kt < N && kt <= vt + kSBufs - 1) {
+            if (kt >= kKStages)
+              ok = mbar_wait(&bar[kBarSFull + (kt - kKStages) % kSBufs], ((kt - kKStages) / kSBufs) & 1,
+                             abort_flag, a.err);
+            if (ok) load_kv(kt++, false);
+          } else {
+            if (vt >= kVStages)
+              ok = mbar_wait(&bar[kBarVEmpty + vt % kVStages], ((vt / kVStages) - 1) & 1, abort_flag, a.err);
+            if (ok) load_kv(vt++, true);
+          }
+        }
+        if (*abort_flag) {  // let copies in flight land before the CTA exits
+          if (N > 0) mbar_wait_drain(&bar[kBarQ], 0);
+          for (int t = (kt > kKStages ? kt - kKStages : 0); t < kt; ++t)
+            mbar_wait_drain(&bar[kBarKFull + t % kKStages], (t / kKStages) & 1);
+          for (int t = (vt > kVStages ? vt - kVStages : 0); t < vt; ++t)
+            mbar_wait_drain(&bar[kBarVFull + t % kVStages], (t / kVStages) & 1);
+        }
+      }
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------ MMA issuer
+      // The whole warp runs the loop, so that the descriptors, addresses and
+      // loop state are warp-uniform values; one elected lane (always the same
+      // one) issues the MMAs and their commits.
+      const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + L::kV), L::kChunkBytes, 1024);
+      constexpr uint64_t kSlotDesc = (uint64_t)(L::kTileBytes >> 4);  // one ring slot
+      const bool leader = elect_one();
+      auto wait_all = [&](uint64_t* b, uint32_t parity) {
+        return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, abort_flag, a.err));
       };
-      if (N > 0) {
-        // the tile's two 64-row halves (a half with no query block reads past
-        // the chunk's rows: zero fill)
-        const int q0 = tile_row(a, bh, m, 0), q1 = tile_row(a, bh, m, 64);
-        const int past = a.d.Fc * a.d.T_pad;
-        mbar_arrive_expect_tx(&bar[kBarQ], L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(smem + L::kQ + c * L::kChunkBytes, &tmQ, &bar[kBarQ], c * 64, q0 < 0 ? past : q0, bh);
-          tma_load_3d(smem + L::kQ + c * L::kChunkBytes + 8192, &tmQ, &bar[kBarQ], c * 64, q1 < 0 ? past : q1, bh);
-        }
-      }
-      // Tile t goes to slot t mod 2 once the tile before it there (t - 2)
-      // was consumed; K and V advance independently.
-      int kt = 0, vt = 0;
-      PollGuard guard;
-      while (kt < N || vt < N) {
-        bool moved = false;
-        if (kt < N && (kt < kStages || mbar_test(&bar[kBarKEmpty + (kt & 1)], ((kt >> 1) - 1) & 1))) {
-          load_kv(kt, false);
-          ++kt;
-          moved = true;
-        }
-        if (vt < N && (vt < kStages || mbar_test(&bar[kBarVEmpty + (vt & 1)], ((vt >> 1) - 1) & 1))) {
-          load_kv(vt, true);
-          ++vt;
-          moved = true;
-        }
-        if (moved) {
-          guard.progress();
-          continue;
-        }
-        if (!guard.idle(abort_flag, a.err)) break;
-        // K(t) frees after S(t - 2), V(t) after PV(t - 2): sleep on the older.
-        if (kt < N && (vt >= N || kt <= vt))
-          mbar_sleep(&bar[kBarKEmpty + (kt & 1)], ((kt >> 1) - 1) & 1, kSleepNs);
-        else
-          mbar_sleep(&bar[kBarVEmpty + (vt & 1)], ((vt >> 1) - 1) & 1, kSleepNs);
-      }
-      if (*abort_flag) {  // let copies in flight land before the CTA exits
-        if (N > 0) mbar_wait_drain(&bar[kBarQ], 0);
-        for (int t = (kt > kStages ? kt - kStages : 0); t < kt; ++t)
-          mbar_wait_drain(&bar[kBarKFull + (t & 1)], (t >> 1) & 1);
-        for (int t = (vt > kStages ? vt - kStages : 0); t < vt; ++t)
-          mbar_wait_drain(&bar[kBarVFull + (t & 1)], (t >> 1) & 1);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t q_addr = smem_u32(smem + L::kQ);
-      const uint32_t k_addr = smem_u32(smem + L::kK);
-      const uint32_t v_addr = smem_u32(smem + L::kV);
-      // S(j) into buffer j mod 2, after PV(j - 2) (which read P(j - 2) from
+      // S(j) into buffer j mod 3, after PV(j - 3) (which read P(j - 3) from
       // that buffer; tcgen05.mma executes in issue order).
       auto issue_score = [&](int j) -> bool {
-        if (!mbar_wait(&bar[kBarKFull + (j & 1)], (j >> 1) & 1, abort_flag, a.err)) return false;
+        const int ks = j % kKStages, sb = j % kSBufs;
+        if (!wait_all(&bar[kBarKFull + ks], (j / kKStages) & 1)) return false;
         tc_fence_after();
-        issue_s<D>(tmem + 128u * (j & 1), q_addr, k_addr + (j & 1) * L::kTileBytes);
-        mma_commit(&bar[kBarSFull + (j & 1)]);
-        mma_commit(&bar[kBarKEmpty + (j & 1)]);
+        if (leader) {
+          issue_s<D>(tmem + kSCol + 128u * sb, q_desc, k_desc + (uint64_t)ks * kSlotDesc);
+          mma_commit(&bar[kBarSFull + sb]);   // S(j) done: also frees K slot j mod 2
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = N > 0 && mbar_wait(&bar[kBarQ], 0, abort_flag, a.err) && issue_score(0);
-      if (ok && N > 1) ok = issue_score(1);
+      bool ok = N > 0 && wait_all(&bar[kBarQ], 0);
+      for (int j = 0; ok && j < kSBufs && j < N; ++j) ok = issue_score(j);
       for (int i = 0; ok && i < N; ++i) {
-        if (!mbar_wait(&bar[kBarPFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err) ||
-            !mbar_wait(&bar[kBarVFull + (i & 1)], (i >> 1) & 1, abort_flag, a.err))
+        const int sb = i % kSBufs;
+        const int vs = i % kVStages;
+        if (!wait_all(&bar[kBarPFull + sb], (i / kSBufs) & 1) ||
+            !wait_all(&bar[kBarVFull + vs], (i / kVStages) & 1))
           break;
         tc_fence_after();
-        // O_even / O_odd: the two softmax warp sets keep separate accumulators
-        issue_pv<D>(tmem + kOCol + 128u * (i & 1), tmem + 128u * (i & 1), v_addr + (i & 1) * L::kTileBytes,
-                    i >= 2);
-        mma_commit(&bar[kBarVEmpty + (i & 1)]);
-        if (i + 1 == N) mma_commit(&bar[kBarODone]);  // O final: the epilogue's wait
-        if (i + 2 < N) ok = issue_score(i + 2);
+        if (leader) {
+          issue_pv<D>(tmem + kOCol, tmem + kSCol + 128u * sb, v_desc + (uint64_t)vs * kSlotDesc, i > 0);
+          mma_commit(&bar[kBarVEmpty + vs]);     // V slot free = PV(i) done
+          if (i + 1 == N) mma_commit(&bar[kBarODone]);  // O final: the epilogue's wait
+        }
+        __syncwarp();
+        if (i + kSBufs < N) ok = issue_score(i + kSBufs);
       }
-      mma_commit(&bar[kBarDrain]);
-      mbar_wait_drain(&bar[kBarDrain], 0);
+      if (leader) {
+        mma_commit(&bar[kBarDrain]);
+        mbar_wait_drain(&bar[kBarDrain], 0);
+      }
+      __syncwarp();
+    } else if (a.kpool_frm) {
+      // ------------------------------------------------------------ spare warps
+      // Frame means of the chunk's new cache frames from their block means
+      // (written by the previous launch), in the order of frame_pool_kernel:
+      // sum_j count_j * mean_j / T_f. CTA i takes frames i, i + grid, ...
+      const Dims& d = a.d;
+      const int nfr = d.B * d.H * d.Fc;
+      const int c0 = tid - (kMmaWarp + 1) * 32;
+      constexpr int kSpare = kAttnThreads - (kMmaWarp + 1) * 32;
+      for (int fr = blockIdx.x; fr < nfr; fr += gridDim.x) {
+        const int fbh = fr / d.Fc;
+        const int f = fr - fbh * d.Fc;
+        const int fslot = (a.t0 + f) % a.W;
+        const float* src = a.kpool_blk + ((size_t)fbh * a.W + fslot) * d.nb * D;
+        float* dst = a.kpool_frm + ((size_t)fbh * a.W + fslot) * D;
+        for (int c = c0; c < D; c += kSpare) {
+          float sum = 0.f;
+          for (int j = 0; j < d.nb; ++j) {
+            const float cnt = (float)((j == d.nb - 1) ? d.tail : d.blk);
+            sum += cnt * src[(size_t)j * D + c];
+          }
+          dst[c] = sum / (float)d.T_f;
+        }
+      }
     }
-  } else if (warp < kSoftmaxWarps) {
+    end_barrier();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  } else {
+    // warpgroups 0 and 1: softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax
     const Dims& d = a.d;
     const int quarter = warp & 3;        // TMEM lane quarter: rows 32 quarter .. + 31
     const int par = warp >> 2;           // this warp's key tiles: par, par + 2, par + 4, ...
     const int r = quarter * 32 + lane;   // query row of the tile = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t ocol = kOCol + 128u * par;  // this warp's O accumulator
     const int mbit = r >> 6;             // this row's bit in a unit mask (warp-uniform)
     // epilogue exchange: (max, sum) [2 parities][128 rows]; flags [2 parities][4 quarters]
     float2* xch = reinterpret_cast<float2*>(smem + L::kRed);
     volatile int* okf = reinterpret_cast<volatile int*>(xch + 2 * 128);
+    // hand-over of the reference maximum: one slot per row, written by the
+    // warp of tile i and read by the warp of tile i + 1 (they alternate)
+    volatile float* hand = reinterpret_cast<volatile float*>(smem + L::kHand);
+    uint64_t* hs_out = &bar[kBarHand + 2 * quarter + par];        // my tiles' maxima
+    uint64_t* hs_in = &bar[kBarHand + 2 * quarter + (par ^ 1)];   // the other warp's
     const float sc = a.scale_log2;
-    float m_used = -INFINITY;  // running maximum in scaled log2 units (possibly stale by < 8)
+    float m_seen = -INFINITY;  // reference maximum (scaled log2 units) l_run is relative to
     float l_run = 0.f;
+    int n_in = 0;              // hand-overs received
     bool ok = true;
     for (int i = par; ok && i < N; i += 2) {
-      const int buf = i & 1;  // = par: S(i) and P(i) live in buffer par
-      ok = mbar_wait(&bar[kBarSFull + buf], (i >> 1) & 1, abort_flag, a.err);
+      const int sb = i % kSBufs;
+      ok = mbar_wait(&bar[kBarSFull + sb], (i / kSBufs) & 1, abort_flag, a.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t sbuf = trow + kSCol + 128u * sb;
       uint32_t s[4][32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tmem_ld32(trow + 128u * buf + 32u * j, s[j]);
+      for (int j = 0; j < 4; ++j) tmem_ld32(sbuf + 32u * j, s[j]);
       const uint32_t e0 = units[2 * i], e1 = units[2 * i + 1];
       const int lim0 = ((e0 >> mbit) & 1u) ? (int)((e0 >> 8) & 0xFFu) : 0;
       const int lim1 = ((e1 >> mbit) & 1u) ? (int)((e1 >> 8) & 0xFFu) : 0;
@@ -515,84 +616,111 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 2; c < 32; c += 2) mx[j] = max3f(mx[j], __uint_as_float(s[j][c]), __uint_as_float(s[j][c + 1]));
       }
       const float mt = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;  // -inf when nothing is valid
-      const bool need = mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt > -INFINITY);
-      if (__any_sync(0xFFFFFFFFu, need)) {
-        const float m_new = need ? mt : m_used;
-        const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
-        if (i >= 2) {
-          // This warp's O holds PV(par .. i-2): S(i) was issued after PV(i-2)
-          // and reported complete, so that PV is done too.
-#pragma unroll 1
-          for (int j = 0; j < D / 16; ++j) {
-            uint32_t o[16];
-            tmem_ld16(trow + ocol + 16u * j, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st16(trow + ocol + 16u * j, o);
-          }
-        }
-        l_run *= alpha;
-        m_used = m_new;
+      // the reference maximum after tile i - 1, from the other warp
+      float m_prev = -INFINITY;
+      if (i > 0) {
+        ok = mbar_wait(hs_in, n_in & 1, abort_flag, a.err);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        m_prev = hand[r];
+        ++n_in;
       }
-      const float base = (m_used == -INFINITY) ? 0.f : m_used;
+      // m only moves up: bring this warp's sum to m_prev, then decide tile i
+      if (m_prev > m_seen) {
+        l_run *= fast_exp2(m_seen - m_prev);   // 0 when m_seen = -inf (l_run is 0 then)
+        m_seen = m_prev;
+      }
+      const bool need = mt > m_prev + kRescaleThreshold || (m_prev == -INFINITY && mt > -INFINITY);
+      const float m_new = need ? mt : m_prev;
+      if (i + 1 < N) {
+        hand[r] = m_new;
+        mbar_arrive(hs_out);
+      }
+      if (need) {
+        l_run *= (m_prev == -INFINITY) ? 0.f : fast_exp2(m_prev - m_new);
+        m_seen = m_new;
+      }
+      const float base = (m_new == -INFINITY) ? 0.f : m_new;
       const float2 sc2 = make_float2(sc, sc);
       const float2 nb2 = make_float2(-base, -base);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      // P = 2^(s sc - m) for the 128 columns, 32 at a time; in a tile without
+      // masked columns (all x finite) a share of the pairs takes the FMA-pipe
+      // polynomial instead of the MUFU, which the two softmax warps of a
+      // scheduler otherwise saturate.
+      auto exp_tile = [&](auto use_poly) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t pk[16];
+        for (int h = 0; h < 4; ++h) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
-                                  sc2, nb2);
-          const float2 p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
-          if (q & 1) acc1 = fadd2(acc1, p);
-          else acc0 = fadd2(acc0, p);
-          pk[q] = cvt_bf16x2(p.x, p.y);
+          for (int q = 0; q < 16; ++q) {
+            const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
+                                    sc2, nb2);
+            float2 p;
+            if (decltype(use_poly)::value && poly_pair(q)) p = exp2_poly2(xv);
+            else p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
+            if (q & 1) acc1 = fadd2(acc1, p);
+            else acc0 = fadd2(acc0, p);
+            pk[q] = cvt_bf16x2(p.x, p.y);
+          }
+          tmem_st16(sbuf + 16u * h, pk);
         }
-        tmem_st16(trow + 128u * buf + 16u * h, pk);
-      }
+      };
+      if (kAttnPoly && full) exp_tile(std::true_type{});
+      else exp_tile(std::false_type{});
       l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      if (__any_sync(0xFFFFFFFFu, need && m_prev > -INFINITY)) {
+        // O holds PV(0 .. i-1) relative to m_prev: rescale the moving rows
+        // once PV(i-1) completed (it frees V slot (i-1) mod 3). PV(i) waits
+        // for this warp's P release below, so O is quiet meanwhile; the
+        // rescale comes after the exponentials, when the scores' registers
+        // are free.
+        ok = mbar_wait(&bar[kBarVEmpty + (i - 1) % kVStages], ((i - 1) / kVStages) & 1, abort_flag, a.err);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float alpha = (need && m_prev > -INFINITY) ? fast_exp2(m_prev - m_new) : 1.f;
+#pragma unroll 1
+        for (int j = 0; j < D / 16; ++j) {
+          uint32_t o[16];
+          tmem_ld16(trow + kOCol + 16u * j, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st16(trow + kOCol + 16u * j, o);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[kBarPFull + buf]);
+      mbar_arrive(&bar[kBarPFull + sb]);
     }
     // ------------------------------------------------------------ epilogue
-    // Both warps of a row range always get here and meet once: the two
-    // partial softmaxes (even and odd key tiles) are merged.
+    // Both warps of a row range always get here and meet once: their sums
+    // (each relative to the maximum it last saw) are merged. O is relative to
+    // the reference after the last tile, the larger of the two maxima.
     bool fin = ok && (N == 0 || mbar_wait(&bar[kBarODone], 0, abort_flag, a.err));  // empty piece: no PV
     fin = __all_sync(0xFFFFFFFFu, fin);
-    xch[par * 128 + r] = make_float2(m_used, l_run);
+    xch[par * 128 + r] = make_float2(m_seen, l_run);
     if (lane == 0) okf[par * 4 + quarter] = fin ? 1 : 0;
     pair_sync(quarter);
     fin = fin && okf[(par ^ 1) * 4 + quarter] != 0;
     if (fin) {
       if (N > 0) tc_fence_after();
-      const float2 e0 = xch[r], e1 = xch[128 + r];  // parities 0 and 1
-      const float M = fmaxf(e0.x, e1.x);
-      const float w0 = (e0.x == -INFINITY) ? 0.f : fast_exp2(e0.x - M);
-      const float w1 = (e1.x == -INFINITY) ? 0.f : fast_exp2(e1.x - M);
-      const float l_tot = e0.y * w0 + e1.y * w1;
-      // this warp writes columns [D/2 par, D/2 par + D/2) from both accumulators
+      const float2 x0 = xch[r], x1 = xch[128 + r];  // parities 0 and 1
+      const float M = fmaxf(x0.x, x1.x);
+      const float w0 = (x0.x == -INFINITY) ? 0.f : fast_exp2(x0.x - M);
+      const float w1 = (x1.x == -INFINITY) ? 0.f : fast_exp2(x1.x - M);
+      const float l_tot = x0.y * w0 + x1.y * w1;
+      // this warp writes columns [D/2 par, D/2 par + D/2)
       const uint32_t c0 = (uint32_t)(D / 2) * par;
-      auto merged = [&](int i, uint32_t (&o)[32]) {  // columns c0 + 32 i .. + 31, relative to M
+      auto load_o = [&](int i, uint32_t (&o)[32]) {  // columns c0 + 32 i .. + 31, relative to M
         if (N == 0) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
           return;
         }
-        uint32_t o1[32];
         tmem_ld32(trow + kOCol + c0 + 32u * i, o);
-        tmem_ld32(trow + kOCol + 128u + c0 + 32u * i, o1);
         tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          // an accumulator no PV wrote (w = 0) holds garbage: never multiply it
-          const float a0 = w0 > 0.f ? __uint_as_float(o[c]) * w0 : 0.f;
-          const float a1 = w1 > 0.f ? __uint_as_float(o1[c]) * w1 : 0.f;
-          o[c] = __float_as_uint(a0 + a1);
-        }
       };
       if (slot >= 0) {
         // A piece of a split tile: O relative to M, M and the sum, for the merge launch.
@@ -600,7 +728,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < D / 64; ++i) {
           uint32_t o[32];
-          merged(i, o);
+          load_o(i, o);
           float4* dst = reinterpret_cast<float4*>(po + 32 * i);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -621,7 +749,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < D / 64; ++i) {
           uint32_t o[32];
-          merged(i, o);
+          load_o(i, o);
           if (row_ok) {
             uint32_t pk[16];
 #pragma unroll
@@ -637,37 +765,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           a.lse[(size_t)bh * d.Lq + n_tok] = (M + log2f(l_tot)) * 0.69314718055994531f;
       }
     }
-  } else if (a.kpool_frm) {
-    // ------------------------------------------------------------ spare warps
-    // Frame means of the chunk's new cache frames from their block means
-    // (written by the previous launch), in the order of frame_pool_kernel:
-    // sum_j count_j * mean_j / T_f. CTA i takes frames i, i + grid, ...
-    const Dims& d = a.d;
-    const int nfr = d.B * d.H * d.Fc;
-    const int c0 = tid - (kMmaWarp + 1) * 32;
-    constexpr int kSpare = kAttnThreads - (kMmaWarp + 1) * 32;
-    for (int fr = blockIdx.x; fr < nfr; fr += gridDim.x) {
-      const int fbh = fr / d.Fc;
-      const int f = fr - fbh * d.Fc;
-      const int fslot = (a.t0 + f) % a.W;
-      const float* src = a.kpool_blk + ((size_t)fbh * a.W + fslot) * d.nb * D;
-      float* dst = a.kpool_frm + ((size_t)fbh * a.W + fslot) * D;
-      for (int c = c0; c < D; c += kSpare) {
-        float sum = 0.f;
-        for (int j = 0; j < d.nb; ++j) {
-          const float cnt = (float)((j == d.nb - 1) ? d.tail : d.blk);
-          sum += cnt * src[(size_t)j * D + c];
-        }
-        dst[c] = sum / (float)d.T_f;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    end_barrier();
   }
 }
 
