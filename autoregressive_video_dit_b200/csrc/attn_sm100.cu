@@ -110,15 +110,15 @@ struct AttnSmem {
   static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
-// Barriers: S buffer b full / P written into it (3 each; S(j) completing also
-// frees K slot j mod 2); K ring slots full (2); V ring slots full and free
-// (3 each; V slot t mod 3
+// Barriers: S buffer b full (3; S(j) completing also frees K slot j mod 2);
+// K ring slots full (2); V ring slots full -- V(t) landed and P(t) written --
+// and free (3 each; V slot t mod 3
 // frees when PV(t) completes, so it also tells that PV(t) is done); Q; O
 // final; one for draining the tensor pipe; the hand-over of the running
 // maximum per row range: [quarter][0] even -> odd tiles, [quarter][1] odd ->
 // even tiles.
-constexpr int kBarSFull = 0, kBarPFull = 3, kBarKFull = 6, kBarVFull = 8, kBarVEmpty = 11,
-              kBarQ = 14, kBarODone = 15, kBarDrain = 16, kBarHand = 17;  // .. 24
+constexpr int kBarSFull = 0, kBarKFull = 3, kBarVFull = 5, kBarVEmpty = 8, kBarQ = 11,
+              kBarODone = 12, kBarDrain = 13, kBarHand = 14;  // .. 21
 
 // Whether full tiles compute a share of their exponentials with the
 // polynomial exp2 (see poly_pair in cva_internal.cuh for the share). Off:
@@ -378,15 +378,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
 
   if (tid == 0) {
-    for (int s = 0; s < kSBufs; ++s) {
-      mbar_init(&bar[kBarSFull + s], 1);
-      mbar_init(&bar[kBarPFull + s], 32 * kSoftmaxWarps / 2);  // one warp set per tile
-    }
+    for (int s = 0; s < kSBufs; ++s) mbar_init(&bar[kBarSFull + s], 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bar[kBarKFull + s], 1);
     }
+    // VFull[s] completes when V(i) landed in slot s AND P(i) was written
+    // (i mod 3 == s for both): the producer's arrive with the byte count plus
+    // the 128 softmax threads of tile i, so the MMA warp waits once per PV.
+    static_assert(kVStages == kSBufs, "V slot and score buffer share an index");
     for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&bar[kBarVFull + s], 1);
+      mbar_init(&bar[kBarVFull + s], 1 + 32 * kSoftmaxWarps / 2);
       mbar_init(&bar[kBarVEmpty + s], 1);
     }
     for (int h = 0; h < 8; ++h) mbar_init(&bar[kBarHand + h], 32);  // one warp's rows
@@ -492,8 +493,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + L::kV), L::kChunkBytes, 1024);
       constexpr uint64_t kSlotDesc = (uint64_t)(L::kTileBytes >> 4);  // one ring slot
       const bool leader = elect_one();
+      const int leader_lane = __ffs(__ballot_sync(0xFFFFFFFFu, leader)) - 1;
+      // Only the issuing lane polls a barrier (32 lanes polling one mbarrier
+      // would serialise on it); the result is broadcast to keep the loop
+      // converged.
       auto wait_all = [&](uint64_t* b, uint32_t parity) {
-        return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, abort_flag, a.err));
+        int r = 1;
+        if (leader) r = mbar_wait(b, parity, abort_flag, a.err) ? 1 : 0;
+        return __shfl_sync(0xFFFFFFFFu, r, leader_lane) != 0;
       };
       // S(j) into buffer j mod 3, after PV(j - 3) (which read P(j - 3) from
       // that buffer; tcgen05.mma executes in issue order).
@@ -513,9 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int i = 0; ok && i < N; ++i) {
         const int sb = i % kSBufs;
         const int vs = i % kVStages;
-        if (!wait_all(&bar[kBarPFull + sb], (i / kSBufs) & 1) ||
-            !wait_all(&bar[kBarVFull + vs], (i / kVStages) & 1))
-          break;
+        if (!wait_all(&bar[kBarVFull + vs], (i / kVStages) & 1)) break;   // V(i) and P(i)
         tc_fence_after();
         if (leader) {
           issue_pv<D>(tmem + kOCol, tmem + kSCol + 128u * sb, v_desc + (uint64_t)vs * kSlotDesc, i > 0);
@@ -692,7 +697,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[kBarPFull + sb]);
+      mbar_arrive(&bar[kBarVFull + sb]);   // P(i) written (sb == V slot of tile i)
     }
     // ------------------------------------------------------------ epilogue
     // Both warps of a row range always get here and meet once: their sums
