@@ -101,7 +101,6 @@ _SIGS = {
                                               c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
     "cva_copy_rows_2d": (c_int32, [c_void_p, c_void_p] + [ctypes.c_int64] * 7 + [c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
-    "cva_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
     "cva_diag_wait_timeout": (c_int32, [c_int32, c_void_p, c_void_p]),
     "cva_kv_cache_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
     "cva_kv_cache_init": (c_int32, [P(KVCache), c_void_p, c_size_t, P(Shape), c_int32, c_int32]),
@@ -219,11 +218,6 @@ def set_stage_events(events) -> None:
         return
     arr = (c_void_p * 4)(*[int(e.cuda_event) for e in events])
     check(lib.cva_set_stage_events(arr, len(events)))
-
-
-def exp2_poly_eval(x, y, stream=None) -> None:
-    """Diagnostic: the softmax's polynomial exp2 on a float32 device tensor."""
-    check(lib.cva_exp2_poly_eval(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
 def diag_wait_timeout(limit_us: int, result, stream=None) -> None:

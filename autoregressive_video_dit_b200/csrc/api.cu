@@ -213,14 +213,6 @@ int cva_set_stage_events(void* const* events, int32_t n) {
   return CVA_OK;
 }
 
-int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream) {
-  if (n < 0) return fail(CVA_EINVAL, "n < 0");
-  if (n == 0) return CVA_OK;
-  if (!x || !y) return fail(CVA_EINVAL, "x or y is NULL");
-  cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "exp2_poly_eval launch");
-}
-
 int cva_diag_wait_timeout(int32_t limit_us, int32_t* result, cva_stream_t stream) {
   if (!result) return fail(CVA_EINVAL, "result is NULL");
   if (!aligned(result, 4)) return fail(CVA_EINVAL, "result must be 4-byte aligned");

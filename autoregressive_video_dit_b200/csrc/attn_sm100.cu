@@ -120,15 +120,6 @@ struct AttnSmem {
 constexpr int kBarSFull = 0, kBarKFull = 3, kBarVFull = 5, kBarVEmpty = 8, kBarQ = 11,
               kBarODone = 12, kBarDrain = 13, kBarHand = 14;  // .. 21
 
-// Whether full tiles compute a share of their exponentials with the
-// polynomial exp2 (see poly_pair in cva_internal.cuh for the share). Off:
-// measured on the 1.3B-shaped dense chunk, every share (1/4 .. 1/2 of the
-// pairs) was slower than the MUFU alone (0.789 ms vs 0.824-0.879 ms).
-#ifndef CVA_ATTN_POLY
-#define CVA_ATTN_POLY 0
-#endif
-constexpr bool kAttnPoly = CVA_ATTN_POLY != 0;
-
 // Above this growth of the row maximum (log2 units) O is rescaled; below
 // it the stale maximum is kept, so P <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
@@ -649,30 +640,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 sc2 = make_float2(sc, sc);
       const float2 nb2 = make_float2(-base, -base);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-      // P = 2^(s sc - m) for the 128 columns, 32 at a time; in a tile without
-      // masked columns (all x finite) a share of the pairs takes the FMA-pipe
-      // polynomial instead of the MUFU, which the two softmax warps of a
-      // scheduler otherwise saturate.
-      auto exp_tile = [&](auto use_poly) {
+      // P = 2^(s sc - m) for the 128 columns, 32 at a time, on the MUFU.
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t pk[16];
+      for (int h = 0; h < 4; ++h) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
-                                    sc2, nb2);
-            float2 p;
-            if (decltype(use_poly)::value && poly_pair(q)) p = exp2_poly2(xv);
-            else p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
-            if (q & 1) acc1 = fadd2(acc1, p);
-            else acc0 = fadd2(acc0, p);
-            pk[q] = cvt_bf16x2(p.x, p.y);
-          }
-          tmem_st16(sbuf + 16u * h, pk);
+        for (int q = 0; q < 16; ++q) {
+          const float2 xv = ffma2(make_float2(__uint_as_float(s[h][2 * q]), __uint_as_float(s[h][2 * q + 1])),
+                                  sc2, nb2);
+          const float2 p = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
+          if (q & 1) acc1 = fadd2(acc1, p);
+          else acc0 = fadd2(acc0, p);
+          pk[q] = cvt_bf16x2(p.x, p.y);
         }
-      };
-      if (kAttnPoly && full) exp_tile(std::true_type{});
-      else exp_tile(std::false_type{});
+        tmem_st16(sbuf + 16u * h, pk);
+      }
       l_run += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       if (__any_sync(0xFFFFFFFFu, need && m_prev > -INFINITY)) {
         // O holds PV(0 .. i-1) relative to m_prev: rescale the moving rows

@@ -331,7 +331,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// ---- packed fp32 arithmetic and the polynomial exp2 -----------------------
+// ---- packed fp32 arithmetic ----------------------------------------------
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -387,38 +387,6 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-// 2^x for a pair of floats on the FMA/ALU pipes instead of the MUFU (Cody and
-// Waite's range reduction): x is clamped to >= -125; adding 1.5 * 2^23 rounds
-// it to the nearest integer n, held in the low mantissa bits of the sum; f =
-// x - n lies in [-1/2, 1/2] and 2^f comes from a degree-3 polynomial fitted
-// for minimum maximum relative error on that interval (7.5e-5; fit_exp2_poly.py
-// in this directory derives the coefficients); n is added to the exponent
-// field. Used for a fixed share of the softmax exponentials so that the MUFU
-// and the FMA pipes share the work.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, make_float2(kShift, kShift));
-  const float2 n = fadd2(t, make_float2(-kShift, -kShift));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(f, make_float2(0.0551716685295105f, 0.0551716685295105f),
-                   make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = ffma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// How many pairs of every 8 in a 64-column page take the polynomial exp2.
-#ifndef CVA_POLY_PAIRS_OF_8
-#define CVA_POLY_PAIRS_OF_8 3
-#endif
-__device__ __forceinline__ constexpr bool poly_pair(int q) {
-  return (CVA_POLY_PAIRS_OF_8 >= 1 && (q & 7) == 7) || (CVA_POLY_PAIRS_OF_8 >= 2 && (q & 7) == 3) ||
-         (CVA_POLY_PAIRS_OF_8 >= 3 && (q & 7) == 5) || (CVA_POLY_PAIRS_OF_8 >= 4 && (q & 7) == 1);
 }
 
 }  // namespace cva

@@ -145,7 +145,6 @@ int check_chunk_call(const void* q, const void* k, const void* v, const cva_kv_c
                      const void* out, size_t* ws_need);
 
 // ---- diagnostics (diag.cu) ------------------------------------------------
-cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_wait_timeout(int* err, int* result, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace cva

@@ -384,13 +384,6 @@ int cva_chunk_attention_noalloc(const void* q, const void* k, const void* v,
  * n must be 4, or 0 with events == NULL to stop. */
 int cva_set_stage_events(void* const* events, int32_t n);
 
-/* Diagnostic: y[i] = the polynomial 2^x[i] the attention softmax evaluates
- * for part of its exponentials on the FMA pipes (Cody-Waite reduction to
- * [-1/2, 1/2], degree-3 minimax polynomial, relative error below 1e-4 for
- * x in [-125, 127]; inputs below -125 are clamped to it). Device buffers of
- * n floats. Not used by the path itself; it lets tests bound the error. */
-int cva_exp2_poly_eval(const float* x, float* y, int32_t n, cva_stream_t stream);
-
 /* Diagnostic of the device-side failure path: one CTA waits, through the
  * bounded wait every pipeline role of the kernels uses, on an mbarrier that
  * nothing arrives at, with a limit of limit_us microseconds (1 .. 10^6)
