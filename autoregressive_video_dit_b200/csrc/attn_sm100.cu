@@ -104,9 +104,9 @@ struct AttnSmem {
   static constexpr int kBytes = kMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
   // While the key list is built, its bitmaps and counts live in the V ring.
-  static constexpr int kBm = kV;                                   // 4 bitmaps
-  static constexpr int kCnt = kBm + 4 * kAttnMaxBitmapWords * 4;   // 3 count arrays
-  static_assert(7 * kAttnMaxBitmapWords * 4 <= kVStages * kTileBytes, "build scratch");
+  static constexpr int kBm = kV;                                   // 2 bitmaps
+  static constexpr int kCnt = kBm + 2 * kAttnMaxBitmapWords * 4;   // word offsets, total
+  static_assert((3 * kAttnMaxBitmapWords + 1) * 4 <= kVStages * kTileBytes, "build scratch");
   static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
@@ -156,26 +156,6 @@ __device__ __forceinline__ int unit_valid(int block_valid, int u) {
   return v < 0 ? 0 : (v > 64 ? 64 : v);
 }
 
-// Tile counts of a key stream (one query tile, or two sharing the stream).
-struct Stream {
-  int TS;    // shared tiles (both lanes)
-  int TA;    // lane A only
-  int TB;    // lane B only
-  int mn;    // min(TA, TB): interleaved pairs
-  __device__ __forceinline__ int total() const { return TS + TA + TB; }
-  __device__ __forceinline__ int tiles_of(int x) const { return TS + (x == 0 ? TA : TB); }
-  // Stream position of lane x's i-th tile.
-  __device__ __forceinline__ int tile_of(int x, int i) const {
-    if (i < TS) return i;
-    const int k = i - TS;
-    return TS + (k < mn ? 2 * k + x : mn + k);
-  }
-  // Entry index of the i-th unit of lane x's private list.
-  __device__ __forceinline__ int private_entry(int x, int i) const {
-    return 2 * tile_of(x, TS + (i >> 1)) + (i & 1);
-  }
-};
-
 // Query block in rows [64 half, 64 half + 64) of tile m of head bh (64-row blocks).
 __device__ __forceinline__ int tile_qb(const AttnArgs& a, int bh, int m, int half) {
   return a.qpair ? a.qpair[((size_t)bh * a.MT + m) * 2 + half] : 2 * m + half;
@@ -187,131 +167,106 @@ __device__ __forceinline__ int tile_row(const AttnArgs& a, int bh, int m, int r)
   return qb < 0 ? -1 : qb * 64 + (r & 63);
 }
 
-// Builds the key stream of the CTA's lanes (tile m0 and, if has_b, m0 + 1)
-// into `ents`; must be called by all threads of the CTA.
-__device__ Stream build_stream(const AttnArgs& a, int m0, bool has_b, int bh, uint32_t* ents,
-                               uint32_t* bm, uint32_t* cnt, int* tot) {
+// Builds the key stream of query tile m0 of head bh into `ents`, two 64-row
+// units per key tile, and returns its number of key tiles; must be called
+// by all threads of the CTA. Dense: the history units, then the current
+// chunk's, padded to a whole tile. Sparse: the current chunk's units padded
+// to a whole tile, then the union of the selected blocks of the tile's two
+// query blocks in ascending order, each unit with a mask of which query
+// block selected it (bit q: rows [64 q, 64 q + 64)). Every thread handles
+// its own list entries and bitmap bits; no step is serial over the list.
+__device__ int build_stream(const AttnArgs& a, int m0, int bh, uint32_t* ents, uint32_t* bm,
+                            uint32_t* cnt) {
   constexpr int kW = kAttnMaxBitmapWords;
   const Dims& d = a.d;
   const int tid = threadIdx.x;
   const int upb = d.blk / 64;
   const int rows64_slot = d.T_pad / 64;
-  const uint32_t all_mask = has_b ? 0xFu : 0x3u;
   const int nbits = a.F * d.nb;
-  const int nw = (nbits + 31) >> 5;
   const bool sparse = a.F > 0 && a.block_idx != nullptr;
-  int nS = (a.F > 0 && !sparse) ? nbits * upb : 0, nA = 0, nB = 0;
-  if (sparse) {
-    for (int i = tid; i < 4 * nw; i += kAttnThreads) bm[(i / nw) * kW + i % nw] = 0u;
-    __syncthreads();
-    const int nq = (d.blk == 64) ? 2 : 1;
-    for (int x = 0; x < (has_b ? 2 : 1); ++x) {
-      for (int q = 0; q < nq; ++q) {
-        const int qb = (d.blk == 64) ? tile_qb(a, bh, m0 + x, q) : m0 + x;
-        if (qb < 0 || qb >= d.NQB) continue;
-        const size_t u = (size_t)bh * d.NQB + qb;
-        int c = a.block_cnt ? a.block_cnt[u] : a.k_b_max;
-        if (c < 0 || c > a.k_b_max) {
-          if (tid == 0) latch_error(a.err, CVA_DEV_BAD_COUNT);
-          c = c < 0 ? 0 : a.k_b_max;
-        }
-        const int32_t* lst = a.block_idx + u * a.k_b_max;
-        uint32_t* row = bm + (2 * x + q) * kW;
-        for (int i = tid; i < c; i += kAttnThreads) {
-          const int id = lst[i];
-          const int rel = id - a.t_lo * d.nb;
-          if (id < 0 || rel < 0 || rel >= nbits) {
-            latch_error(a.err, CVA_DEV_BAD_INDEX);
-            continue;
-          }
-          atomicOr(&row[rel >> 5], 1u << (rel & 31));
-          if (nq == 1) atomicOr(&row[kW + (rel >> 5)], 1u << (rel & 31));  // both bits of the lane
-        }
-      }
-    }
-    __syncthreads();
-    for (int w = tid; w < nw; w += kAttnThreads) {
-      const uint32_t ia = bm[w] | bm[kW + w], ib = bm[2 * kW + w] | bm[3 * kW + w];
-      cnt[w] = __popc(ia & ib) * upb;
-      cnt[kW + w] = __popc(ia & ~ib) * upb;
-      cnt[2 * kW + w] = __popc(ib & ~ia) * upb;
-    }
-    __syncthreads();
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < 3) {  // exclusive scan of class `warp`'s per-word counts
-      uint32_t* c = cnt + warp * kW;
-      int carry = 0;
-      for (int base = 0; base < nw; base += 32) {
-        const int w = base + lane;
-        const int v = (w < nw) ? (int)c[w] : 0;
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        if (w < nw) c[w] = (uint32_t)(carry + incl - v);
-        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-      if (lane == 0) tot[warp] = carry;
-    }
-    __syncthreads();
-    nS = tot[0];
-    nA = tot[1];
-    nB = tot[2];
-  }
   const int cur = d.Fc * d.nb * upb;
-  Stream st;
-  st.TS = (nS + cur + 1) >> 1;
-  st.TA = (nA + 1) >> 1;
-  st.TB = (nB + 1) >> 1;
-  st.mn = st.TA < st.TB ? st.TA : st.TB;
-  if (a.F > 0 && !sparse) {
-    for (int i = tid; i < nS; i += kAttnThreads) {
-      const int br = i / upb, u = i - br * upb;
-      const int fp = br / d.nb, j = br - fp * d.nb;
-      const int slot = (a.t_lo + fp) % a.W;
-      const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-      ents[i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), all_mask);
-    }
-  } else if (sparse) {
-    for (int w = tid; w < nw; w += kAttnThreads) {
-      const uint32_t b0 = bm[w], b1 = bm[kW + w], b2 = bm[2 * kW + w], b3 = bm[3 * kW + w];
-      const uint32_t ia = b0 | b1, ib = b2 | b3;
-      uint32_t any = ia | ib;
-      int pos[3] = {(int)cnt[w], (int)cnt[kW + w], (int)cnt[2 * kW + w]};
-      while (any) {
-        const int bit = __ffs(any) - 1;
-        any &= any - 1u;
-        const int cls = ((ia >> bit) & 1u) ? (((ib >> bit) & 1u) ? 0 : 1) : 2;
-        const int rel = w * 32 + bit;
-        const int fp = rel / d.nb, j = rel - fp * d.nb;
-        const int slot = (a.t_lo + fp) % a.W;
-        const uint32_t mask = ((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1) | (((b2 >> bit) & 1u) << 2) |
-                              (((b3 >> bit) & 1u) << 3);
-        const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-        for (int u = 0; u < upb; ++u) {
-          const int i = cls == 0 ? pos[0]++ : (cls == 1 ? pos[1]++ : pos[2]++);
-          const int e = cls == 0 ? i : st.private_entry(cls - 1, i);
-          ents[e] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
-        }
-      }
-    }
+  const int hist = (a.F > 0 && !sparse) ? nbits * upb : 0;   // dense history units
+  const int c0 = sparse ? 0 : hist;                          // first unit of the current chunk
+  for (int i = tid; i < hist; i += kAttnThreads) {
+    const int br = i / upb, u = i - br * upb;
+    const int fp = br / d.nb, j = br - fp * d.nb;
+    const int slot = (a.t_lo + fp) % a.W;
+    const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+    ents[i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 0x3u);
   }
   for (int i = tid; i < cur; i += kAttnThreads) {
     const int br = i / upb, u = i - br * upb;
     const int f = br / d.nb, j = br - f * d.nb;
     const int slot = (a.t0 + f) % a.W;
     const int vb = (j == d.nb - 1) ? d.tail : d.blk;
-    ents[nS + i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), all_mask);
+    ents[c0 + i] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), 0x3u);
   }
-  if (tid == 0) {
-    if ((nS + cur) & 1) ents[2 * st.TS - 1] = 0u;
-    if (nA & 1) ents[st.private_entry(0, nA)] = 0u;
-    if (nB & 1) ents[st.private_entry(1, nB)] = 0u;
+  if (tid == 0 && ((c0 + cur) & 1)) ents[c0 + cur] = 0u;
+  const int lead = (c0 + cur + 1) >> 1;   // key tiles before the sparse section
+  if (!sparse) {
+    __syncthreads();
+    return lead;
+  }
+  const int nw = (nbits + 31) >> 5;
+  const int nq = (d.blk == 64) ? 2 : 1;
+  const int kbm = a.k_b_max;
+  for (int i = tid; i < 2 * kW; i += kAttnThreads) bm[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < nq * kbm; i += kAttnThreads) {
+    const int q = i >= kbm ? 1 : 0;
+    const int k = i - q * kbm;
+    const int qb = (d.blk == 64) ? tile_qb(a, bh, m0, q) : m0;
+    if (qb < 0 || qb >= d.NQB) continue;
+    const size_t u = (size_t)bh * d.NQB + qb;
+    const int id = a.block_idx[u * kbm + k];   // in the list's storage whatever the count
+    int c = a.block_cnt ? a.block_cnt[u] : kbm;
+    if (c < 0 || c > kbm) {
+      if (k == 0) latch_error(a.err, CVA_DEV_BAD_COUNT);
+      c = c < 0 ? 0 : kbm;
+    }
+    if (k >= c) continue;
+    const int rel = id - a.t_lo * d.nb;
+    if (id < 0 || rel < 0 || rel >= nbits) {
+      latch_error(a.err, CVA_DEV_BAD_INDEX);
+      continue;
+    }
+    atomicOr(&bm[q * kW + (rel >> 5)], 1u << (rel & 31));
   }
   __syncthreads();
-  return st;
+  if (tid < 32) {  // exclusive scan of the units per bitmap word
+    int carry = 0;
+    for (int base = 0; base < nw; base += 32) {
+      const int w = base + tid;
+      const int v = (w < nw) ? __popc(bm[w] | bm[kW + w]) * upb : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (tid >= o) incl += t;
+      }
+      if (w < nw) cnt[w] = (uint32_t)(carry + incl - v);
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (tid == 0) cnt[kW] = (uint32_t)carry;
+  }
+  __syncthreads();
+  const int n_sp = (int)cnt[kW];
+  uint32_t* sp = ents + 2 * lead;
+  for (int rel = tid; rel < nbits; rel += kAttnThreads) {
+    const int w = rel >> 5, bit = rel & 31;
+    const uint32_t b0 = bm[w], b1 = bm[kW + w], any = b0 | b1;
+    if (!((any >> bit) & 1u)) continue;
+    const int pos = (int)cnt[w] + __popc(any & ((1u << bit) - 1u)) * upb;
+    const uint32_t mask = nq == 1 ? 0x3u : (((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1));
+    const int fp = rel / d.nb, j = rel - fp * d.nb;
+    const int slot = (a.t_lo + fp) % a.W;
+    const int vb = (j == d.nb - 1) ? d.tail : d.blk;
+    for (int u = 0; u < upb; ++u)
+      sp[pos + u] = make_unit(slot * rows64_slot + j * upb + u, unit_valid(vb, u), mask);
+  }
+  if (tid == 0 && (n_sp & 1)) sp[n_sp] = 0u;
+  __syncthreads();
+  return lead + ((n_sp + 1) >> 1);
 }
 
 // The MMAs of one key tile, from shared-memory descriptors computed once per
@@ -365,7 +320,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  int* tot = reinterpret_cast<int*>(smem + L::kMisc + 8);  // 3 ints
   uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L::kEnt);
 
   if (tid == 0) {
@@ -392,9 +346,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  const Stream st = build_stream(a, m, false, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
-                                 reinterpret_cast<uint32_t*>(smem + L::kCnt), tot);
-  const int NT = st.total();  // key tiles of the tile, in stream order
+  // key tiles of the tile, in stream order
+  const int NT = build_stream(a, m, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
+                              reinterpret_cast<uint32_t*>(smem + L::kCnt));
   // This work item's key tiles: all, or piece `piece` of `pieces`.
   const int i_lo = slot < 0 ? 0 : (int)((int64_t)NT * piece / a.pieces);
   const int N = slot < 0 ? NT : (int)((int64_t)NT * (piece + 1) / a.pieces) - i_lo;

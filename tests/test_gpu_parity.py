@@ -439,6 +439,59 @@ def test_c3_hsa_end_to_end_sampled(ops, chunk):
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean, rel)
 
 
+def _ws_pairs(wl, ws, k_f, k_b):
+    """The query-block pair table the fused call wrote into its workspace
+    (after the counts in the layout of cva_chunk_workspace_bytes)."""
+    d = wl
+    bhq = d.B * d.H * d.NQB
+    r256 = lambda x: (x + 255) // 256 * 256
+    o_p = (r256(d.B * d.H * d.Fc * d.T_pad * d.D * 2) + r256(bhq * d.D * 4) + r256(bhq * max(k_f, 0) * 4)
+           + r256(bhq * max(k_b, 0) * 4) + r256(bhq * 4))
+    MT = -(-d.Fc * d.T_pad // 128)
+    raw = ws.cpu().numpy()
+    return raw[o_p:o_p + d.B * d.H * MT * 8].view(np.int32).reshape(d.B * d.H, MT, 2)
+
+
+def _mutual_best_pairs(frames):
+    """Rounds: every unpaired query block names the unpaired block sharing the
+    most picked frames (31 or more count as equal), ties to the lower index;
+    blocks naming each other pair up; a last lone block pairs with none (-1).
+    Pairs in order of their lower block."""
+    sets = [set(int(t) for t in f) for f in frames]
+    n = len(sets)
+    ov = lambda i, j: min(len(sets[i] & sets[j]), 31)
+    free, partner = set(range(n)), {}
+    while len(free) >= 2:
+        best = {}
+        for i in free:
+            best[i] = max((j for j in free if j != i), key=lambda j: (ov(i, j), -j))
+        for i in free:
+            if best[i] > i and best[best[i]] == i:
+                partner[i], partner[best[i]] = best[i], i
+        free -= set(partner)
+    return [(i, partner[i]) if i in partner else (i, -1) for i in range(n) if partner.get(i, n) > i]
+
+
+def test_query_block_pairs_are_mutual_best(ops):
+    # c3 chunk 7: 18 history frames, 8 picked per query block, so the fused
+    # call pairs the 64-row query blocks by shared frames before the attention
+    wl = WORKLOADS["c3"].with_chunk(7)
+    res, cache = _gpu_stream(ops, wl, 7)
+    out, ws, k_f, k_b = res[7]
+    _, F = cache.history_frames(wl.t0_of(7))
+    kfe = min(k_f, F)
+    assert wl.blk == 64 and F >= 2 * kfe
+    fr, _, _ = ws_lists(wl, ws, k_f, k_b, kfe)
+    fr = fr.reshape(wl.B * wl.H, wl.NQB, kfe)
+    got = _ws_pairs(wl, ws, k_f, k_b)
+    for bh in range(wl.B * wl.H):
+        want = _mutual_best_pairs(fr[bh])
+        assert [tuple(int(v) for v in p) for p in got[bh, :len(want)]] == want, bh
+        assert (got[bh, len(want):] == -1).all()
+        ids = sorted(v for p in want for v in p if v >= 0)
+        assert ids == list(range(wl.NQB))
+
+
 def test_c4_end_to_end_sampled(ops):
     wl = WORKLOADS["c4"]
     heads = [0, 21, 39]
