@@ -3,16 +3,17 @@
 // history frames are picked with frame-pooled keys, then the important
 // blocks inside those frames with block-pooled keys.
 //
-// Four warps per (batch*head, query block), four query blocks of a head
-// to a CTA (so that they share the pooled keys in L1), with no barrier
-// wider than a query block's four warps: the work of a query block is a
+// P warps per (batch*head, query block) -- four, two or one, as many as
+// keep every query block of the call resident at once -- and 16 / P query
+// blocks of a head to a CTA (so that they share the pooled keys in L1),
+// with no barrier wider than a query block's warps: the work of a query block is a
 // chain of dependent steps (load, score, pick, load, score, pick), so its
 // latency is what counts. Scores are dot products of the block-pooled
 // query with pooled keys, 32 at a time per warp: each lane forms the
 // partial dot products of its D/32 slice for 32 candidates, and a
 // reduce-scatter through warp shuffles (31 exchanges) leaves candidate
-// base+i's score on lane i; the four warps share the candidate groups of
-// the second level. Every candidate becomes a 64-bit key (order-preserving
+// base+i's score on lane i; the query block's warps share the candidate
+// groups of the second level. Every candidate becomes a 64-bit key (order-preserving
 // score bits, then the complement of its position), so keys are distinct
 // and "ranks by score, ties toward the lower position" is their descending
 // order. The k-th largest key is found by a radix select over the key
@@ -33,9 +34,8 @@
 
 namespace cva {
 
-constexpr int kSelQbs = 4;                   // query blocks per CTA
-constexpr int kSelWarpsPerQb = 4;
-constexpr int kSelThreads = 32 * kSelWarpsPerQb * kSelQbs;
+constexpr int kSelThreads = 512;             // 16 warps: 16 / P query blocks of P warps
+constexpr int kSelSmSlots = 32;              // warps per SM at the kernel's 64 registers
 constexpr int kSelMaxFrames = 256;
 
 __device__ __forceinline__ uint32_t ordered_bits(float s) {
@@ -195,28 +195,37 @@ inline size_t sel_group_bytes(int nmax, bool topp) {
   return (b + 15) & ~size_t(15);
 }
 
-template <int D>
+template <int D, int P>
 __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a, int nmax, int units,
-                                                                   int group_bytes) {
+                                                                      int group_bytes) {
   extern __shared__ __align__(16) uint8_t sel_smem[];
+  constexpr int kQbs = kSelThreads / (32 * P);  // query blocks per CTA
+  constexpr int kGT = 32 * P;                   // threads per query block
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = warp / kSelWarpsPerQb;       // query block of the CTA
-  const int wq = warp - g * kSelWarpsPerQb;  // warp within it
-  const int gt = 32 * wq + lane;             // thread within it
-  constexpr int kGT = 32 * kSelWarpsPerQb;
+  const int g = warp / P;       // query block of the CTA
+  const int wq = warp - g * P;  // warp within it
+  const int gt = 32 * wq + lane;
   const Dims& d = a.d;
-  const int u = blockIdx.x * kSelQbs + g;
-  if (u >= units) return;  // the query block's four warps together
-  // named barrier 1 + g over the query block's warps (immediate ids, so that
-  // the kernel holds five barriers, not sixteen)
+  const int u = blockIdx.x * kQbs + g;
+  if (u >= units) return;  // the query block's warps together
+  // barrier over the query block's warps: the warp itself, or named barrier
+  // 1 + g (immediate ids, so that the kernel holds only the ids it uses)
   auto gsync = [g] {
-    static_assert(kSelQbs == 4, "one case per query block");
-    switch (g) {
-      case 0: asm volatile("bar.sync 1, %0;" ::"n"(kGT) : "memory"); break;
-      case 1: asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory"); break;
-      case 2: asm volatile("bar.sync 3, %0;" ::"n"(kGT) : "memory"); break;
-      default: asm volatile("bar.sync 4, %0;" ::"n"(kGT) : "memory"); break;
+    static_assert(P == 1 || P == 2 || P == 4, "warps per query block");
+    if constexpr (P == 1) {
+      __syncwarp();
+    } else {
+      switch (g) {
+        case 0: asm volatile("bar.sync 1, %0;" ::"n"(kGT) : "memory"); break;
+        case 1: asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory"); break;
+        case 2: asm volatile("bar.sync 3, %0;" ::"n"(kGT) : "memory"); break;
+        case 3: asm volatile("bar.sync 4, %0;" ::"n"(kGT) : "memory"); break;
+        case 4: asm volatile("bar.sync 5, %0;" ::"n"(kGT) : "memory"); break;
+        case 5: asm volatile("bar.sync 6, %0;" ::"n"(kGT) : "memory"); break;
+        case 6: asm volatile("bar.sync 7, %0;" ::"n"(kGT) : "memory"); break;
+        default: asm volatile("bar.sync 8, %0;" ::"n"(kGT) : "memory"); break;
+      }
     }
   };
   const int bh = u / d.NQB;
@@ -274,7 +283,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
   }
   gsync();
 
-  // ---- level 2: blocks of the chosen frames (all four warps) -----------------
+  // ---- level 2: blocks of the chosen frames (all the query block's warps) ----
   const int C = kfe * d.nb;
   const int kb = a.k_b;
   for (int c = gt; c < C; c += kGT) {
@@ -305,7 +314,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
     smax = warp_max(smax);
     if (lane == 0) red[wq] = smax;
     gsync();
-    smax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    smax = red[0];
+#pragma unroll
+    for (int w = 1; w < P; ++w) smax = fmaxf(smax, red[w]);
     const float tail = (float)d.tail;
     float part = 0.f;
     for (int c = gt; c < C; c += kGT) {
@@ -317,7 +328,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
     part = warp_sum(part);
     if (lane == 0) red[4 + wq] = part;
     gsync();
-    thresh = a.topp * ((red[4] + red[5]) + (red[6] + red[7]));
+    float total = red[4];
+#pragma unroll
+    for (int w = 1; w < P; ++w) total += red[4 + w];
+    thresh = a.topp * total;
     // take flags over the row offsets, which the scoring no longer needs
     for (int c = gt; c < C; c += kGT) {
       float above;
@@ -496,24 +510,41 @@ cudaError_t launch_pair_query_blocks(const int32_t* frame_idx, int kfe, const Di
   return cudaGetLastError();
 }
 
+template <int D, int P>
+static cudaError_t launch_select_p(const SelectArgs& a, int nmax, int units, size_t gb, cudaStream_t stream) {
+  constexpr int qbs = kSelThreads / (32 * P);
+  const size_t smem = gb * qbs;
+  cudaError_t e = cudaFuncSetAttribute(hsa_select_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  hsa_select_kernel<D, P><<<(units + qbs - 1) / qbs, kSelThreads, smem, stream>>>(a, nmax, units, (int)gb);
+  return cudaGetLastError();
+}
+
+// Warps per query block: as many as keep every query block resident at
+// once (the work of one is a latency chain that more warps shorten), and
+// as shared memory allows.
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   const int kfe = a.k_f < a.F ? a.k_f : a.F;
   const int nmax = a.F > kfe * a.d.nb ? a.F : kfe * a.d.nb;
   const size_t gb = sel_group_bytes(nmax, a.topp > 0.f);
-  const size_t smem = gb * kSelQbs;
   const int units = a.d.B * a.d.H * a.d.NQB;
-  dim3 grid((units + kSelQbs - 1) / kSelQbs);
-  cudaError_t e;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t smem_cap = 100 * 1024;  // two CTAs per SM
+  int P = 4;
+  while (P > 1 && (int64_t)sms * kSelSmSlots / P < units) P >>= 1;
+  while (P < 4 && gb * (kSelThreads / (32 * P)) > smem_cap) P <<= 1;
+  if (gb * (kSelThreads / (32 * P)) > smem_cap * 2) return cudaErrorInvalidValue;
   if (a.d.D == 128) {
-    e = cudaFuncSetAttribute(hsa_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    hsa_select_kernel<128><<<grid, kSelThreads, smem, stream>>>(a, nmax, units, (int)gb);
-  } else {
-    e = cudaFuncSetAttribute(hsa_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    hsa_select_kernel<64><<<grid, kSelThreads, smem, stream>>>(a, nmax, units, (int)gb);
+    if (P == 4) return launch_select_p<128, 4>(a, nmax, units, gb, stream);
+    if (P == 2) return launch_select_p<128, 2>(a, nmax, units, gb, stream);
+    return launch_select_p<128, 1>(a, nmax, units, gb, stream);
   }
-  return cudaGetLastError();
+  if (P == 4) return launch_select_p<64, 4>(a, nmax, units, gb, stream);
+  if (P == 2) return launch_select_p<64, 2>(a, nmax, units, gb, stream);
+  return launch_select_p<64, 1>(a, nmax, units, gb, stream);
 }
 
 }  // namespace cva
