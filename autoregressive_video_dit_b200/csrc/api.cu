@@ -507,9 +507,11 @@ int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk
 
 // Selection launch; topp > 0 switches the second level to the top-p budget
 // with cap k_b.
+// dependent: the launch directly follows the chunk's rotation kernel on the
+// stream (programmatic dependent launch).
 static int select_impl(const float* qpool_blk, const cva_kv_cache* cache, int t0, int k_f, int k_b,
                        int32_t* frame_idx, int32_t* block_idx, int32_t* block_cnt, int k_b_max,
-                       float topp, cudaStream_t s) {
+                       float topp, cudaStream_t s, bool dependent = false) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -544,7 +546,7 @@ static int select_impl(const float* qpool_blk, const cva_kv_cache* cache, int t0
     }
     return CVA_OK;
   }
-  cudaError_t e = launch_select(a, s);
+  cudaError_t e = launch_select(a, s, dependent);
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "hsa_select launch");
 }
 
@@ -600,7 +602,7 @@ static int sm_count() {
 // block per tile), when fewer than 2 k_f history frames leave little to pair,
 // or beyond the pairing's limits (tiles then hold blocks 2m and 2m+1).
 static int pair_impl(const Dims& d, const cva_kv_cache* cache, int t0, int k_f, const int32_t* fidx,
-                     int32_t* qpair_ws, const int32_t** qpair, cudaStream_t s) {
+                     int32_t* qpair_ws, const int32_t** qpair, cudaStream_t s, bool dependent) {
   *qpair = nullptr;
   if (d.blk != 64) return CVA_OK;
   int t_lo, F;
@@ -610,7 +612,7 @@ static int pair_impl(const Dims& d, const cva_kv_cache* cache, int t0, int k_f, 
   // with at least twice as many history frames as picks.
   if (F == 0 || kfe < 1 || F < 2 * kfe) return CVA_OK;
   const int MT = (d.Fc * d.T_pad + 127) / 128;
-  cudaError_t e = launch_pair_query_blocks(fidx, kfe, d, t_lo, F, MT, qpair_ws, s);
+  cudaError_t e = launch_pair_query_blocks(fidx, kfe, d, t_lo, F, MT, qpair_ws, s, dependent);
   if (e == cudaErrorInvalidValue) return CVA_OK;  // beyond the pairing's limits: default tiles
   if (e != cudaSuccess) return cuda_fail(e, "pair_query_blocks launch");
   *qpair = qpair_ws;
@@ -622,7 +624,7 @@ static int pair_impl(const Dims& d, const cva_kv_cache* cache, int t0, int k_f, 
 static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const int32_t* block_idx,
                      const int32_t* block_cnt, int k_b_max, void* out, float* lse, void* split_ws,
                      size_t split_bytes, cudaStream_t s, bool frame_means = false,
-                     const int32_t* qpair = nullptr) {
+                     const int32_t* qpair = nullptr, bool dependent = false) {
   const Dims d = make_dims(cache->shape);
   int t_lo, F;
   history(cache, t0, &t_lo, &F);
@@ -666,7 +668,7 @@ static int attn_impl(const void* q_rot, const cva_kv_cache* cache, int t0, const
     }
   }
   const char* why = "";
-  cudaError_t e = launch_attention(a, q_rot, cache->k, cache->v, s, &why);
+  cudaError_t e = launch_attention(a, q_rot, cache->k, cache->v, s, &why, dependent);
   if (e == cudaErrorInvalidValue && why[0]) return fail(CVA_ELAUNCH, "attention: %s", why);
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "blocksparse_attn_fwd launch");
 }
@@ -719,6 +721,9 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   int32_t* bcnt = reinterpret_cast<int32_t*>(ws + w.block_cnt);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool sparse = !dense && F > 0;
+  // Each kernel after the first one follows one of this call's kernels:
+  // programmatic dependent launches, unless stage events sit between them.
+  const bool chain = !g_stage_on;
   cudaError_t e = stage_mark(0, s);
   if (e != cudaSuccess) return cuda_fail(e, "stage event");
   // steps 1-3: projection, rotation, append and pooling in the fused kernel
@@ -727,14 +732,14 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   const int32_t* qpair = nullptr;
   if (sparse) {
-    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, 0.f, s);
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, 0.f, s, chain);
     if (rc) return rc;
-    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s);
+    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s, chain);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair, chain);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;
@@ -899,19 +904,21 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
   if (e != cudaSuccess) return cuda_fail(e, "chunk_attention rope/append launch");
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "stage event");
 
-  // step 4
+  // step 4; each kernel from here on follows one of this call's kernels:
+  // programmatic dependent launches, unless stage events sit between them
   const bool sparse = !dense && F > 0;
+  const bool chain = !g_stage_on;
   const int32_t* qpair = nullptr;
   if (sparse) {
-    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, topp, s);
+    rc = select_impl(qpool, cache, t0, k_f, k_b, fidx, bidx, bcnt, k_b, topp, s, chain);
     if (rc) return rc;
-    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s);
+    rc = pair_impl(d, cache, t0, k_f, fidx, reinterpret_cast<int32_t*>(ws + w.qpair), &qpair, s, chain);
     if (rc) return rc;
   }
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   // step 5 (with the frame means of the new cache frames)
   rc = attn_impl(q_rot, cache, t0, sparse ? bidx : nullptr, sparse ? bcnt : nullptr,
-                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair);
+                 sparse ? k_b : 0, out, lse, ws + w.attn, attn_split_bytes(d), s, true, qpair, chain);
   if (rc) return rc;
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "stage event");
   return CVA_OK;

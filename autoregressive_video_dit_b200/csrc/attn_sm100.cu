@@ -304,6 +304,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  griddep_launch_dependents();
   // Work item: a whole tile, or one key-range piece of a tail tile.
   int tile = blockIdx.x, piece = 0, slot = -1;
   if (tile >= a.Qf) {
@@ -346,6 +347,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  griddep_wait();  // block lists, pairs and Q come from the preceding kernels
   // key tiles of the tile, in stream order
   const int NT = build_stream(a, m, bh, ents, reinterpret_cast<uint32_t*>(smem + L::kBm),
                               reinterpret_cast<uint32_t*>(smem + L::kCnt));
@@ -716,6 +718,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // columns each).
 template <int D>
 __global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a) {
+  griddep_wait();  // the pieces come from the attention launch
   const Dims& d = a.d;
   const int tt = blockIdx.x / kBM;      // split tile among the tail
   const int r = blockIdx.x - tt * kBM;  // row of the tile
@@ -801,7 +804,7 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
 
 template <int D>
 static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
-                                      const CUtensorMap& mv, cudaStream_t stream) {
+                                      const CUtensorMap& mv, cudaStream_t stream, bool dependent) {
   using L = AttnSmem<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::kAlloc);
@@ -810,15 +813,14 @@ static cudaError_t launch_attention_d(const AttnArgs& a, const CUtensorMap& mq, 
   if (e != cudaSuccess) return e;
   const int tiles = a.MT * a.d.B * a.d.H;
   dim3 grid(a.Qf + (tiles - a.Qf) * a.pieces);
-  attn_fwd_kernel<D><<<grid, kAttnThreads, L::kAlloc, stream>>>(mq, mk, mv, a);
-  e = cudaGetLastError();
+  e = launch_kernel(attn_fwd_kernel<D>, grid, dim3(kAttnThreads), L::kAlloc, stream, dependent, mq, mk, mv, a);
   if (e != cudaSuccess || a.Qf == tiles) return e;
-  attn_merge_kernel<D><<<(tiles - a.Qf) * kBM, D / 4, 0, stream>>>(a);
-  return cudaGetLastError();
+  // the merge always follows the attention launch
+  return launch_kernel(attn_merge_kernel<D>, dim3((tiles - a.Qf) * kBM), dim3(D / 4), 0, stream, true, a);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
-                             const void* cache_v, cudaStream_t stream, const char** why) {
+                             const void* cache_v, cudaStream_t stream, const char** why, bool dependent) {
   const Dims& d = a.d;
   CUtensorMap mq, mk, mv;
   const uint64_t bh = (uint64_t)d.B * d.H;
@@ -828,8 +830,8 @@ cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* c
     *why = "cuTensorMapEncodeTiled failed (driver entry point or tensor shape)";
     return cudaErrorInvalidValue;
   }
-  return d.D == 128 ? launch_attention_d<128>(a, mq, mk, mv, stream)
-                    : launch_attention_d<64>(a, mq, mk, mv, stream);
+  return d.D == 128 ? launch_attention_d<128>(a, mq, mk, mv, stream, dependent)
+                    : launch_attention_d<64>(a, mq, mk, mv, stream, dependent);
 }
 
 }  // namespace cva

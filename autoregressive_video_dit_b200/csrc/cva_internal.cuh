@@ -75,6 +75,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch. A kernel of the fused chunk call that
+// follows another of this library's kernels on the stream is launched so
+// that it may be scheduled while its predecessor drains; it calls
+// griddep_wait() before it reads or writes memory that earlier work touches
+// (the wait returns once the predecessor grid has completed and its writes
+// are visible, at once when the launch was an ordinary one). Every kernel
+// of the chain calls griddep_launch_dependents() on entry, which lets its
+// successor be scheduled once all of its own CTAs are resident.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }

@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
   const int wq = warp - g * P;  // warp within it
   const int gt = 32 * wq + lane;
   const Dims& d = a.d;
+  griddep_launch_dependents();
   const int u = blockIdx.x * kQbs + g;
   if (u >= units) return;  // the query block's warps together
   // barrier over the query block's warps: the warp itself, or named barrier
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
       asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
     }
   }
+  griddep_wait();  // the pooled queries come from the preceding rotation
   float q[D / 32];
   {
     const float* qp = a.qpool + (size_t)u * D + lane * (D / 32);
@@ -394,6 +396,8 @@ __global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const i
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = tid;  // the block this thread speaks for
+  griddep_launch_dependents();
+  griddep_wait();  // the frame lists come from the preceding selection
   if (i < NQB) {
     uint32_t m[kPairWords] = {};
     const int32_t* fr = frame_idx + ((size_t)bh * NQB + i) * kfe;
@@ -499,32 +503,33 @@ __global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const i
 }
 
 cudaError_t launch_pair_query_blocks(const int32_t* frame_idx, int kfe, const Dims& d, int t_lo, int F, int MT,
-                                     int32_t* qpair, cudaStream_t stream) {
+                                     int32_t* qpair, cudaStream_t stream, bool dependent) {
   if (d.NQB > kPairMaxQB || F > kSelMaxFrames || kfe < 1 || kfe > 255) return cudaErrorInvalidValue;
   const int L = kfe + 1 < kPairLevels ? kfe + 1 : kPairLevels;
   const size_t smem = (size_t)d.NQB * L * 16;
   cudaError_t e = cudaFuncSetAttribute(pair_query_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  pair_query_blocks_kernel<<<d.B * d.H, kPairThreads, smem, stream>>>(frame_idx, kfe, d.NQB, t_lo, F, MT, qpair);
-  return cudaGetLastError();
+  return launch_kernel(pair_query_blocks_kernel, dim3(d.B * d.H), dim3(kPairThreads), smem, stream, dependent,
+                       frame_idx, kfe, d.NQB, t_lo, F, MT, qpair);
 }
 
 template <int D, int P>
-static cudaError_t launch_select_p(const SelectArgs& a, int nmax, int units, size_t gb, cudaStream_t stream) {
+static cudaError_t launch_select_p(const SelectArgs& a, int nmax, int units, size_t gb, cudaStream_t stream,
+                                   bool dependent) {
   constexpr int qbs = kSelThreads / (32 * P);
   const size_t smem = gb * qbs;
   cudaError_t e = cudaFuncSetAttribute(hsa_select_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  hsa_select_kernel<D, P><<<(units + qbs - 1) / qbs, kSelThreads, smem, stream>>>(a, nmax, units, (int)gb);
-  return cudaGetLastError();
+  return launch_kernel(hsa_select_kernel<D, P>, dim3((units + qbs - 1) / qbs), dim3(kSelThreads), smem, stream,
+                       dependent, a, nmax, units, (int)gb);
 }
 
 // Warps per query block: as many as keep every query block resident at
 // once (the work of one is a latency chain that more warps shorten), and
 // as shared memory allows.
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream, bool dependent) {
   const int kfe = a.k_f < a.F ? a.k_f : a.F;
   const int nmax = a.F > kfe * a.d.nb ? a.F : kfe * a.d.nb;
   const size_t gb = sel_group_bytes(nmax, a.topp > 0.f);
@@ -538,13 +543,13 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   while (P < 4 && gb * (kSelThreads / (32 * P)) > smem_cap) P <<= 1;
   if (gb * (kSelThreads / (32 * P)) > smem_cap * 2) return cudaErrorInvalidValue;
   if (a.d.D == 128) {
-    if (P == 4) return launch_select_p<128, 4>(a, nmax, units, gb, stream);
-    if (P == 2) return launch_select_p<128, 2>(a, nmax, units, gb, stream);
-    return launch_select_p<128, 1>(a, nmax, units, gb, stream);
+    if (P == 4) return launch_select_p<128, 4>(a, nmax, units, gb, stream, dependent);
+    if (P == 2) return launch_select_p<128, 2>(a, nmax, units, gb, stream, dependent);
+    return launch_select_p<128, 1>(a, nmax, units, gb, stream, dependent);
   }
-  if (P == 4) return launch_select_p<64, 4>(a, nmax, units, gb, stream);
-  if (P == 2) return launch_select_p<64, 2>(a, nmax, units, gb, stream);
-  return launch_select_p<64, 1>(a, nmax, units, gb, stream);
+  if (P == 4) return launch_select_p<64, 4>(a, nmax, units, gb, stream, dependent);
+  if (P == 2) return launch_select_p<64, 2>(a, nmax, units, gb, stream, dependent);
+  return launch_select_p<64, 1>(a, nmax, units, gb, stream, dependent);
 }
 
 }  // namespace cva

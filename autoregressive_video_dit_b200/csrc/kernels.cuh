@@ -5,6 +5,25 @@
 
 namespace cva {
 
+// Launches `kernel`; with `dependent`, as a programmatic dependent launch
+// (the kernel must call griddep_wait() before it touches memory that the
+// previous work on the stream reads or writes).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, bool dependent, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- steps 1-3: rotary embedding, cache append, pooling (rope_pool.cu) ----
 enum : int { kTokenMajor = 0, kHeadMajor = 1, kCacheSlots = 2 };
 enum : int { kPoolNone = 0, kPoolChunk = 1, kPoolCache = 2 };
@@ -59,11 +78,11 @@ struct SelectArgs {
   float topp;
   float temp_log2;         // log2(e) / sqrt(D)
 };
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream, bool dependent = false);
 // Pairs each head's 64-row query blocks into 128-row attention tiles by the
 // overlap of their picked frames (hsa_select.cu).
 cudaError_t launch_pair_query_blocks(const int32_t* frame_idx, int kfe, const Dims& d, int t_lo, int F,
-                                     int MT, int32_t* qpair, cudaStream_t stream);
+                                     int MT, int32_t* qpair, cudaStream_t stream, bool dependent = false);
 
 // ---- step 5: attention (attn_sm100.cu) -----------------------------------
 struct AttnArgs {
@@ -99,7 +118,8 @@ constexpr int kAttnMaxBitmapWords = 256;  // history blocks per CTA <= 8192
 
 // Builds the tensor maps and launches the attention kernel.
 cudaError_t launch_attention(const AttnArgs& a, const void* q_rot, const void* cache_k,
-                             const void* cache_v, cudaStream_t stream, const char** why);
+                             const void* cache_v, cudaStream_t stream, const char** why,
+                             bool dependent = false);
 
 // Tiled TMA descriptor of a bf16 tensor [d2][d1][d0] (d0 innermost) with a
 // box of 64 x box1 elements and 128-byte swizzle (attn_sm100.cu).

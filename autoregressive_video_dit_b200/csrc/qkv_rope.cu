@@ -81,6 +81,7 @@ __device__ __forceinline__ void qkv_group_sync(int g) {  // the 4 warps of colum
 __global__ void __launch_bounds__(kQkvThreads, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const QkvArgs a) {
+  griddep_launch_dependents();
   using L = QkvSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

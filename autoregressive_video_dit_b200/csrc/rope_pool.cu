@@ -117,6 +117,7 @@ __device__ __forceinline__ void warp_col_sums(const float (&acc)[8], float* red,
 // at least MINB CTAs per SM.
 template <int D, int NJ, int FL, int ROWS, int MINB>
 __global__ void __launch_bounds__(256, MINB) rope_pool_kernel(RopePoolArgs a) {
+  griddep_launch_dependents();
   constexpr int kCG = D / 8;         // column groups (16-byte vectors) per row
   constexpr int kRP = 256 / kCG;     // rows per pass
   constexpr int kPass = ROWS / kRP;  // passes per batch
@@ -312,6 +313,7 @@ __global__ void __launch_bounds__(256, 3)
     rope_pool_tma_kernel(const __grid_constant__ CUtensorMap m0, const __grid_constant__ CUtensorMap m1,
                          const __grid_constant__ CUtensorMap m2, const __grid_constant__ CUtensorMap mt,
                          RopePoolArgs a) {
+  griddep_launch_dependents();
   using L = RopeTma<D>;
   constexpr int kCG = D / 8;
   constexpr int kRP = 256 / kCG;

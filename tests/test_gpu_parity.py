@@ -492,6 +492,31 @@ def test_query_block_pairs_are_mutual_best(ops):
         assert ids == list(range(wl.NQB))
 
 
+def test_back_to_back_launches_match_staged_launches(ops):
+    # Without stage events the fused call lets each kernel start while the
+    # previous one drains (each waits for its inputs on the device); with
+    # them, the kernels run one after another. The outputs are the same bits.
+    import torch
+    wl = WORKLOADS["c3"].with_chunk(7)
+    res, cache = _gpu_stream(ops, wl, 7)
+    out_chain, ws, k_f, k_b = res[7]
+    x = inputs(wl, 7, 0, None, key_centres(wl, 0) if wl.keys == "clustered" else None)
+    tabs = _tables(ops, wl, 0)
+    out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in evs:
+        e.record()   # creates the underlying event
+    ops.set_stage_events(evs)
+    try:
+        ops.chunk_attention(to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]), cache, tabs, wl.t0_of(7),
+                            k_f, k_b, ws, out)
+        torch.cuda.synchronize()
+    finally:
+        ops.set_stage_events(None)
+    assert ops.device_status() == 0
+    assert np.array_equal(from_dev(out), out_chain)
+
+
 def test_c4_end_to_end_sampled(ops):
     wl = WORKLOADS["c4"]
     heads = [0, 21, 39]
