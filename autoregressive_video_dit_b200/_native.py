@@ -71,6 +71,9 @@ _SIGS = {
     "cva_rope3d_precompute_tokens": (c_int32, [P(RopeCfg), c_void_p]),
     "cva_rope3d_apply": (c_int32, [c_void_p, c_void_p, P(RopeTables), P(Shape), c_int32, c_int32, c_void_p]),
     "cva_kv_append": (c_int32, [c_void_p, c_void_p, P(KVCache), P(RopeTables), c_int32, c_void_p]),
+    "cva_rotate_append_pool": (c_int32, [c_void_p, c_void_p, c_void_p, P(KVCache), P(RopeTables), c_int32,
+                                         c_void_p, c_void_p, c_void_p]),
+    "cva_kv_frame_means": (c_int32, [P(KVCache), c_int32, c_void_p]),
     "cva_history_frames": (c_int32, [P(KVCache), c_int32, P(c_int32), P(c_int32)]),
     "cva_qkv_rope_append": (c_int32, [c_void_p, c_void_p, c_int32, P(KVCache), P(RopeTables), c_int32,
                                       c_void_p, c_void_p, c_void_p]),
@@ -300,6 +303,19 @@ def kv_append(k, v, cache: DeviceKVCache, tables: Optional[DeviceRopeTables], t0
     check(lib.cva_kv_append(_ptr(k), _ptr(v), ctypes.byref(cache.struct),
                             None if tables is None else ctypes.byref(tables.struct), t0,
                             _stream(stream)))
+
+
+def rotate_append_pool(q, k, v, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, q_rot,
+                       qpool_blk=None, stream=None) -> None:
+    """Steps 1-3 of chunk_attention in its single launch (see cva.h); the frame
+    means of the new frames come from kv_frame_means or chunk_attention."""
+    check(lib.cva_rotate_append_pool(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cache.struct),
+                                     ctypes.byref(tables.struct), t0, _ptr(q_rot), _ptr(qpool_blk),
+                                     _stream(stream)))
+
+
+def kv_frame_means(cache: DeviceKVCache, t0: int, stream=None) -> None:
+    check(lib.cva_kv_frame_means(ctypes.byref(cache.struct), t0, _stream(stream)))
 
 
 def qkv_rope_append(x, w_qkv, cache: DeviceKVCache, tables: DeviceRopeTables, t0: int, q_rot,

@@ -505,6 +505,30 @@ int cva_hsa_compress(const void* q_rot, const cva_shape* shape, float* qpool_blk
   return CVA_OK;
 }
 
+// Arguments of the rotate/append/pool launch of steps 1-3: Q rotated into
+// q_rot (head-major, frames padded to whole blocks) with its block means in
+// qpool (when not NULL), K rotated and V copied into the cache slots of the
+// chunk's frames with the block means of the stored keys.
+static RopePoolArgs chunk_rope_args(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                                    const cva_rope_tables* tables, int32_t t0, uint16_t* q_rot,
+                                    float* qpool) {
+  const Dims d = make_dims(cache->shape);
+  RopePoolArgs a = {};
+  a.job[0] = {static_cast<const uint16_t*>(q), kTokenMajor, q_rot, kHeadMajor, 1, qpool,
+              qpool ? (int)kPoolChunk : (int)kPoolNone};
+  a.job[1] = {static_cast<const uint16_t*>(k), kTokenMajor, static_cast<uint16_t*>(cache->k),
+              kCacheSlots, 1, cache->kpool_blk, kPoolCache};
+  a.job[2] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
+              kCacheSlots, 0, nullptr, kPoolNone};
+  a.njobs = 3;
+  a.err = device_error_word();
+  a.tab = make_tab(tables, d.D);
+  a.d = d;
+  a.t0 = t0;
+  a.W = cache->window;
+  return a;
+}
+
 // Selection launch; topp > 0 switches the second level to the top-p budget
 // with cap k_b.
 // dependent: the launch directly follows the chunk's rotation kernel on the
@@ -745,6 +769,34 @@ int cva_chunk_attention_qkv(const void* x, const void* w_qkv, int32_t hidden, co
   return CVA_OK;
 }
 
+int cva_rotate_append_pool(const void* q, const void* k, const void* v, const cva_kv_cache* cache,
+                           const cva_rope_tables* tables, int32_t t0, void* q_rot, float* qpool_blk,
+                           cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!q || !k || !v || !q_rot) return fail(CVA_EINVAL, "NULL buffer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q_rot, 16))
+    return fail(CVA_EINVAL, "q, k, v and q_rot must be 16-byte aligned");
+  if (qpool_blk && !aligned(qpool_blk, 16)) return fail(CVA_EINVAL, "qpool_blk must be 16-byte aligned");
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  const Dims d = make_dims(cache->shape);
+  rc = check_tables(tables, d, t0);
+  if (rc) return rc;
+  const RopePoolArgs a = chunk_rope_args(q, k, v, cache, tables, t0, static_cast<uint16_t*>(q_rot), qpool_blk);
+  cudaError_t e = launch_rope_pool(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "rotate_append_pool launch");
+}
+
+int cva_kv_frame_means(const cva_kv_cache* cache, int32_t t0, cva_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (t0 < cache->t_begin) return fail(CVA_ERANGE, "t0 %d before the stream start %d", t0, cache->t_begin);
+  const Dims d = make_dims(cache->shape);
+  FramePoolArgs fp = {cache->kpool_blk, cache->kpool_frm, kPoolCache, d, t0, cache->window};
+  cudaError_t e = launch_frame_pool(fp, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "kv_frame_means launch");
+}
+
 int cva_copy_rows_2d(const void* src, void* dst, int64_t n0, int64_t n1, int64_t inner_bytes,
                      int64_t src_stride0, int64_t src_stride1, int64_t dst_stride0, int64_t dst_stride1,
                      cva_stream_t stream) {
@@ -885,19 +937,7 @@ static int chunk_attention_impl(const void* q, const void* k, const void* v, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // steps 1-3: rotate Q (+ block pools) and K (+ append, block pools), copy V
-  RopePoolArgs a = {};
-  a.job[0] = {static_cast<const uint16_t*>(q), kTokenMajor, q_rot, kHeadMajor, 1,
-              dense ? nullptr : qpool, dense ? (int)kPoolNone : (int)kPoolChunk};
-  a.job[1] = {static_cast<const uint16_t*>(k), kTokenMajor, static_cast<uint16_t*>(cache->k),
-              kCacheSlots, 1, cache->kpool_blk, kPoolCache};
-  a.job[2] = {static_cast<const uint16_t*>(v), kTokenMajor, static_cast<uint16_t*>(cache->v),
-              kCacheSlots, 0, nullptr, kPoolNone};
-  a.njobs = 3;
-  a.err = device_error_word();
-  a.tab = make_tab(tables, d.D);
-  a.d = d;
-  a.t0 = t0;
-  a.W = cache->window;
+  const RopePoolArgs a = chunk_rope_args(q, k, v, cache, tables, t0, q_rot, dense ? nullptr : qpool);
   cudaError_t e = stage_mark(0, s);
   if (e != cudaSuccess) return cuda_fail(e, "stage event");
   e = launch_rope_pool(a, s);

@@ -374,6 +374,44 @@ def time_steps(step, flush, n, stream, stages=True):
             [e[1].elapsed_time(e[2]) for e in st_ev], [e[2].elapsed_time(e[3]) for e in st_ev])
 
 
+def rope_kernel_ms(st, rounds=10, sets=4):
+    """Per-launch time (ms) of the rotate/append/pool launch alone, through
+    its own entry point: `sets` input sets with their own outputs (q_rot,
+    pooled queries, and the slots of distinct frames of a scratch cache), in
+    total larger than L2, launched back to back round-robin between two
+    events on the current stream (each launch reads inputs that three other
+    launches' traffic has evicted)."""
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    wl = st["wl"]
+    cache = ops.DeviceKVCache(st["shape"], wl.window, 0)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    shp = (wl.B, wl.Lq, wl.H, wl.D)
+    sets_ = []
+    for i in range(sets):
+        q, k, v = (torch.randn(shp, generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+        q_rot = torch.empty(wl.B * wl.H * wl.Fc * wl.T_pad * wl.D, dtype=torch.bfloat16, device="cuda")
+        qpool = torch.empty(wl.B * wl.H * wl.NQB * wl.D, dtype=torch.float32, device="cuda")
+        sets_.append((q, k, v, q_rot, qpool, max(0, wl.t0 - wl.Fc * i)))
+
+    def launch(x):
+        ops.rotate_append_pool(x[0], x[1], x[2], cache, st["tables"], x[5], x[3], x[4])
+
+    for x in sets_:
+        launch(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(rounds):
+        for x in sets_:
+            launch(x)
+    e1.record()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    return e0.elapsed_time(e1) / (rounds * sets)
+
+
 def reduce_over_ranks(ms, work, device):
     """Weak scaling over independent instances: the job takes as long as its
     slowest rank (max of `ms`) and does the sum of the ranks' `work`. With
@@ -473,8 +511,9 @@ def measure_chunk(args, wl, layer, stream, flush, n, clocks_on, world=1):
         dist.barrier()
     clocks = sampler.stop()
     assert ops.device_status() == 0
+    rope_k = rope_kernel_ms(st)   # after the timed region, on a scratch cache
     return dict(st=st, step=step, flops=flops, step_ms=step_ms, rope_ms=rope_ms, sel_ms=sel_ms,
-                attn_ms=attn_ms, staged_ms=staged_ms, clocks=clocks)
+                attn_ms=attn_ms, staged_ms=staged_ms, rope_kernel_ms=rope_k, clocks=clocks)
 
 
 def attention_peak(peaks, clocks):
@@ -491,7 +530,8 @@ def config_entry(m, peaks, peak_src):
     st, wl = m["st"], m["st"]["wl"]
     ms = statistics.mean(m["step_ms"])
     attn = statistics.mean(m["attn_ms"])
-    rope = statistics.mean(m["rope_ms"])
+    rope = m["rope_kernel_ms"]
+    rope_stage = statistics.mean(m["rope_ms"])
     sel = statistics.mean(m["sel_ms"])
     peak, kind = attention_peak(peaks, m["clocks"])
     ach = m["flops"] / (attn * 1e-3) / 1e12
@@ -504,12 +544,16 @@ def config_entry(m, peaks, peak_src):
         "attention_ms": attn, "attention_tflops": ach,
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": ach, "peak": peak,
                      "unit": "TFLOP/s", "frac": ach / peak,
-                     "peak_source": f"{peak_src} {kind}", "flops": "useful: each query block's own keys"},
+                     "peak_source": f"{peak_src} {kind}", "flops": "useful: each query block's own keys",
+                     "traffic": recorded_traffic("attn_sm100.cu", wl.key)},
         "rotate_append_pool_us": 1e3 * rope,
+        "rotate_append_pool_stage_us": 1e3 * rope_stage,
         "roofline_hbm": {"kernel": "rope_pool_tma_kernel", "bound": "hbm",
                          "achieved": rb / (rope * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": rb / (rope * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
-                         "algorithmic_bytes": rb},
+                         "algorithmic_bytes": rb,
+                         "timing": "per launch of its own entry point, 40 launches back to back over "
+                                   "4 input sets larger than L2, CUDA events"},
         "select_us": 1e3 * sel, "select_share": sel / statistics.mean(m["staged_ms"]),
         "ms_stage_pass": statistics.mean(m["staged_ms"]),
         "steps": len(m["step_ms"]), "stat": "mean", "clocks": m["clocks"],
@@ -607,7 +651,7 @@ def run_cuda(args):
         "latency_ms": ms_max,
         "attention_tflop_per_chunk": flops / 1e12,
         "frac_of_bf16_peak": (total_flops / world) / (ms_max * 1e-3) / 1e12 / entry["roofline"]["peak"],
-        "stage_ms": {"rotate_append_pool": entry["rotate_append_pool_us"] * 1e-3,
+        "stage_ms": {"rotate_append_pool": entry["rotate_append_pool_stage_us"] * 1e-3,
                      "select": entry["select_us"] * 1e-3, "attention": entry["attention_ms"],
                      "step_with_stage_events": entry["ms_stage_pass"],
                      "note": "a separate pass with events between the stages (kernels then launch "

@@ -324,6 +324,30 @@ int cva_chunk_attention_topp(const void* q, const void* k, const void* v,
                              int32_t t0, int32_t k_f, int32_t k_cap, float p, void* workspace,
                              size_t ws_bytes, void* out, float* lse, cva_stream_t stream);
 
+/* Steps 1-3 of cva_chunk_attention alone, in its single launch ("Light
+ * Forcing" section 2.2 token compression and the global time index of
+ * section 2B of the Causal-RoPE page): Q rotated with global time t0 into
+ * q_rot and, when qpool_blk is not NULL, its block means; K rotated and V
+ * copied into the cache slots of frames t0 .. t0+Fc-1 (rolling eviction as
+ * cva_kv_append), with the block means of the stored keys. The frame means
+ * of the new frames are not written: cva_chunk_attention writes them in its
+ * attention launch, and cva_kv_frame_means writes them for callers that
+ * run their own attention.
+ *   q, k, v: bf16 [B, Lq, H, D] (16-byte aligned);
+ *   q_rot: bf16 [B][H][Fc*T_pad][D] (out_layout 1 of cva_rope3d_apply);
+ *   qpool_blk: fp32 [B][H][NQB][D] or NULL.
+ * tables must hold the per-position table (cva_rope3d_precompute_tokens).
+ * Errors as cva_chunk_attention's. */
+int cva_rotate_append_pool(const void* q, const void* k, const void* v,
+                           const cva_kv_cache* cache, const cva_rope_tables* tables,
+                           int32_t t0, void* q_rot, float* qpool_blk, cva_stream_t stream);
+
+/* Frame means (fp32, over each frame's T_f tokens, fixed order) of the
+ * cached keys of frames t0 .. t0+Fc-1 from their block means ("Light
+ * Forcing" section 2.2: frame-pooled keys); completes cva_rotate_append_pool
+ * for callers that do not follow it with cva_chunk_attention. */
+int cva_kv_frame_means(const cva_kv_cache* cache, int32_t t0, cva_stream_t stream);
+
 /* Steps 1-5 for one chunk starting from the hidden states: the fused QKV
  * projection with Causal-RoPE, append and pooling (cva_qkv_rope_append, the
  * pages' section 2C operator fusion), then selection with (k_f, k_b)

@@ -517,6 +517,40 @@ def test_back_to_back_launches_match_staged_launches(ops):
     assert np.array_equal(from_dev(out), out_chain)
 
 
+@pytest.mark.parametrize("key", ["r64", "c1s"])
+def test_rotate_append_pool_is_the_fused_calls_first_launch(ops, key):
+    # steps 1-3 alone (plus the frame means) leave the same q_rot, pooled
+    # queries and cache contents as the fused call's first launch
+    import torch
+    wl = WORKLOADS[key]
+    shp = shape_of(wl)
+    tabs = _tables(ops, wl)
+    x = inputs(wl, 1, 0, None, key_centres(wl, 0) if wl.keys == "clustered" else None)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    fused = ops.DeviceKVCache(shp, wl.window, 0)
+    ws = torch.zeros(ops.chunk_workspace_bytes(shp, -1, 0), dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    ops.chunk_attention(q, k, v, fused, tabs, wl.t0_of(1), -1, 0, ws, out)
+    staged = ops.DeviceKVCache(shp, wl.window, 0)
+    n_qrot = wl.B * wl.H * wl.Fc * wl.T_pad * wl.D
+    q_rot = torch.empty(n_qrot, dtype=torch.bfloat16, device="cuda")
+    qpool = torch.empty(wl.B * wl.H * wl.NQB * wl.D, dtype=torch.float32, device="cuda")
+    ops.rotate_append_pool(q, k, v, staged, tabs, wl.t0_of(1), q_rot, qpool)
+    ops.kv_frame_means(staged, wl.t0_of(1))
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert torch.equal(q_rot, ws[:n_qrot * 2].view(torch.bfloat16))
+    for a, b in ((staged.k, fused.k), (staged.v, fused.v), (staged.kpool_blk, fused.kpool_blk)):
+        assert torch.equal(a, b)
+    torch.testing.assert_close(staged.kpool_frm, fused.kpool_frm, rtol=1e-6, atol=1e-6)
+    # the dense first chunk does not pool its queries; the staged step-3 entry
+    # pools the same rotated queries
+    ref = torch.empty_like(qpool)
+    ops.hsa_compress(q_rot, shp, ref)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(qpool, ref, rtol=1e-6, atol=1e-6)
+
+
 def test_c4_end_to_end_sampled(ops):
     wl = WORKLOADS["c4"]
     heads = [0, 21, 39]
