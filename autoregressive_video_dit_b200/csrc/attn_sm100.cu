@@ -727,20 +727,43 @@ __global__ void __launch_bounds__(D / 4) attn_merge_kernel(const AttnArgs a) {
   const int m = tile - bh * a.MT;
   const int s0 = tt * a.pieces;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+  // One pass over the pieces, eight at a time (their loads independent of
+  // one another): the running maximum M and the sums rescaled when it grows.
   float M = -INFINITY;
-  for (int p = 0; p < a.pieces; ++p) M = fmaxf(M, ml[(size_t)(s0 + p) * kBM + r].x);
   float lsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const int c = 4 * threadIdx.x;
-  for (int p = 0; p < a.pieces; ++p) {
-    const float2 e = ml[(size_t)(s0 + p) * kBM + r];
-    const float w = (e.x == -INFINITY) ? 0.f : exp2f(e.x - M);
-    lsum += w * e.y;
-    const float4 o = *reinterpret_cast<const float4*>(a.part_o + ((size_t)(s0 + p) * kBM + r) * D + c);
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
+  for (int p0 = 0; p0 < a.pieces; p0 += 8) {
+    float2 e[8];
+    float4 o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const size_t row = (size_t)(s0 + p0 + j) * kBM + r;
+      const bool in = p0 + j < a.pieces;
+      e[j] = in ? ml[row] : make_float2(-INFINITY, 0.f);
+      o[j] = in ? *reinterpret_cast<const float4*>(a.part_o + row * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float bm = M;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) bm = fmaxf(bm, e[j].x);
+    if (bm > M) {
+      const float sc = (M == -INFINITY) ? 0.f : exp2f(M - bm);
+      lsum *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+      M = bm;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float w = (e[j].x == -INFINITY) ? 0.f : exp2f(e[j].x - M);
+      lsum += w * e[j].y;
+      acc.x += w * o[j].x;
+      acc.y += w * o[j].y;
+      acc.z += w * o[j].z;
+      acc.w += w * o[j].w;
+    }
   }
   const int pr = tile_row(a, bh, m, r);
   if (pr < 0) return;
