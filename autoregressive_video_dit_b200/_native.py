@@ -105,6 +105,7 @@ _SIGS = {
     "cva_copy_rows_2d": (c_int32, [c_void_p, c_void_p] + [ctypes.c_int64] * 7 + [c_void_p]),
     "cva_set_stage_events": (c_int32, [P(c_void_p), c_int32]),
     "cva_diag_wait_timeout": (c_int32, [c_int32, c_void_p, c_void_p]),
+    "cva_diag_mma_cycles": (c_int32, [c_int32, c_int32, c_int32, c_void_p, c_int32, c_void_p]),
     "cva_kv_cache_bytes": (c_int32, [P(Shape), c_int32, P(c_size_t)]),
     "cva_kv_cache_init": (c_int32, [P(KVCache), c_void_p, c_size_t, P(Shape), c_int32, c_int32]),
     "cva_cag_budget": (c_int32, [P(CagCfg), c_int32, c_int32, c_int32, P(c_int32), P(c_int32)]),
@@ -221,6 +222,12 @@ def set_stage_events(events) -> None:
         return
     arr = (c_void_p * 4)(*[int(e.cuda_event) for e in events])
     check(lib.cva_set_stage_events(arr, len(events)))
+
+
+def diag_mma_cycles(m: int, n: int, iters: int, cycles, stream=None) -> None:
+    """Diagnostic: clock64 span of iters x 4 back-to-back m x n x 16 MMAs per
+    CTA, one CTA per element of the uint64 (int64) device tensor `cycles`."""
+    check(lib.cva_diag_mma_cycles(m, n, iters, _ptr(cycles), cycles.numel(), _stream(stream)))
 
 
 def diag_wait_timeout(limit_us: int, result, stream=None) -> None:

@@ -35,6 +35,18 @@ int cuda_fail(cudaError_t e, const char* where) {
   return fail(CVA_ELAUNCH, "%s: %s", where, cudaGetErrorString(e));
 }
 
+// SMs of the current device (cached per device).
+static int sm_count() {
+  static int counts[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 // Device error word, one per device; kernels receive its address.
 __device__ int g_dev_err;
 
@@ -221,6 +233,22 @@ int cva_diag_wait_timeout(int32_t limit_us, int32_t* result, cva_stream_t stream
   if (!err) return fail(CVA_ELAUNCH, "device error word unavailable");
   cudaError_t e = launch_wait_timeout(err, result, (uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CVA_OK : cuda_fail(e, "diag_wait_timeout launch");
+}
+
+int cva_diag_mma_cycles(int32_t m, int32_t n, int32_t iters, uint64_t* cycles, int32_t ctas,
+                        cva_stream_t stream) {
+  if (!cycles) return fail(CVA_EINVAL, "cycles is NULL");
+  if (!aligned(cycles, 8)) return fail(CVA_EINVAL, "cycles must be 8-byte aligned");
+  if (m != 64 && m != 128) return fail(CVA_EINVAL, "m must be 64 or 128");
+  if (n < 8 || n > 256 || n % (m == 64 ? 8 : 16)) return fail(CVA_EINVAL, "n must be a multiple of %d in [8, 256]", m == 64 ? 8 : 16);
+  if (iters < 1 || iters > 65536) return fail(CVA_EINVAL, "iters must lie in [1, 65536]");
+  const int nsm = sm_count();
+  if (ctas < 1 || (nsm > 0 && ctas > nsm)) return fail(CVA_EINVAL, "ctas must lie in [1, SM count]");
+  int* err = device_error_word();
+  if (!err) return fail(CVA_ELAUNCH, "device error word unavailable");
+  cudaError_t e = launch_mma_cycles(m, n, iters, reinterpret_cast<unsigned long long*>(cycles), ctas, err,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CVA_OK : cuda_fail(e, "diag_mma_cycles launch");
 }
 
 int cva_rope_axis_pairs(int32_t head_dim, int32_t* p_t, int32_t* p_h, int32_t* p_w) {
@@ -607,18 +635,6 @@ int cva_attn_workspace_bytes(const cva_shape* shape, int32_t k_b_max, size_t* by
   (void)k_b_max;
   *bytes = attn_split_bytes(make_dims(*shape));
   return CVA_OK;
-}
-
-// SMs of the current device (cached per device).
-static int sm_count() {
-  static int counts[128] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
-  if (counts[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) counts[dev] = n;
-  }
-  return counts[dev];
 }
 
 // Tiles of two 64-row query blocks paired by their picked frames (the fused

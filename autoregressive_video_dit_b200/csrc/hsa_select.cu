@@ -243,13 +243,23 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsa_select_kernel(SelectArgs a
   const float* kblk = a.kpool_blk + (size_t)bh * a.W * d.nb * D;
   const int F = a.F;
   {
-    // L2 prefetch of this query block's share of the head's history block
-    // means (128-byte lines; the head's query blocks take every NQB-th line).
-    const int lpf = d.nb * D / 32;  // lines per frame
+    // L2 prefetch of this query block's share of the head's history frame
+    // and block means (128-byte lines; the head's query blocks take every
+    // NQB-th line). No kernel of the call writes them, so this may run
+    // before the wait for the preceding launch.
     const int r = u - bh * d.NQB;
-    for (int l = r + d.NQB * gt; l < F * lpf; l += kGT * d.NQB) {
-      const int p = l / lpf;
-      const float* line = kblk + (size_t)((a.t_lo + p) % a.W) * d.nb * D + (size_t)(l - p * lpf) * 32;
+    const int lpf = d.nb * D / 32;  // block-mean lines per frame
+    constexpr int kFrmLines = D / 32;
+    for (int l = r + d.NQB * gt; l < F * (lpf + kFrmLines); l += kGT * d.NQB) {
+      const float* line;
+      if (l < F * lpf) {
+        const int p = l / lpf;
+        line = kblk + (size_t)((a.t_lo + p) % a.W) * d.nb * D + (size_t)(l - p * lpf) * 32;
+      } else {
+        const int lf = l - F * lpf;
+        const int p = lf / kFrmLines;
+        line = kfrm + (size_t)((a.t_lo + p) % a.W) * D + (size_t)(lf - p * kFrmLines) * 32;
+      }
       asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
     }
   }
@@ -420,35 +430,52 @@ __global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const i
   // whether the overlap occurs. Each item is a short dependent chain, so the
   // items are spread over all 32 warps.
   for (int r = warp; r < NQB; r += kPairThreads / 32) {
+    // the four 32-block groups as independent chains
+    int ov[4];
+    bool valid[4];
+#pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int j = 32 * k + lane;
-      const bool valid = j < NQB && j != r;
-      int ov = 0;
-      if (valid) {
-        for (int w = 0; w < nw; ++w) ov += __popc(mask[w][r] & mask[w][j]);
-        ov = ov < L - 1 ? ov : L - 1;
+      valid[k] = j < NQB && j != r;
+      int o = 0;
+      if (valid[k]) {
+        for (int w = 0; w < nw; ++w) o += __popc(mask[w][r] & mask[w][j]);
+        o = o < L - 1 ? o : L - 1;
       }
-      uint32_t word = __ballot_sync(0xFFFFFFFFu, valid);
-#pragma unroll
-      for (int bit = 0; bit < 5; ++bit) {
-        const uint32_t bb = __ballot_sync(0xFFFFFFFFu, (ov >> bit) & 1);
-        word &= ((lane >> bit) & 1) ? bb : ~bb;
-      }
-      if (lane < L) lvl[(r * L + lane) * 4 + k] = word;
-      const uint32_t occ = __ballot_sync(0xFFFFFFFFu, lane < L && word != 0u);
-      if (lane == 0 && occ) atomicOr(&occurs[r], occ);
+      ov[k] = o;
     }
+    uint32_t word[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) word[k] = __ballot_sync(0xFFFFFFFFu, valid[k]);
+#pragma unroll
+    for (int bit = 0; bit < 5; ++bit) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t bb = __ballot_sync(0xFFFFFFFFu, (ov[k] >> bit) & 1);
+        word[k] &= ((lane >> bit) & 1) ? bb : ~bb;
+      }
+    }
+    if (lane < L) {
+      uint4 wv = make_uint4(word[0], word[1], word[2], word[3]);
+      reinterpret_cast<uint4*>(lvl)[r * L + lane] = wv;
+    }
+    const uint32_t occ = __ballot_sync(0xFFFFFFFFu, lane < L && (word[0] | word[1] | word[2] | word[3]) != 0u);
+    if (lane == 0) occurs[r] = occ;
   }
   if (tid < kPairMaxQB && lane == 0) {
     const int lo = 32 * warp;
     freew[warp] = NQB >= lo + 32 ? 0xFFFFFFFFu : (NQB > lo ? (1u << (NQB - lo)) - 1u : 0u);
   }
   __syncthreads();
+  // The rounds involve one thread per query block: warps 0-3, with their
+  // own named barrier; the other warps are done.
+  if (tid >= kPairMaxQB) return;
+  auto qsync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kPairMaxQB) : "memory"); };
   int nfree = NQB;
   // every round pairs at least two blocks, so NQB / 2 rounds suffice
   for (int round = 0; nfree >= 2 && round < kPairMaxQB / 2; ++round) {
     const uint32_t f0 = freew[0], f1 = freew[1], f2 = freew[2], f3 = freew[3];
-    const uint32_t mine = warp == 0 ? f0 : (warp == 1 ? f1 : (warp == 2 ? f2 : (warp == 3 ? f3 : 0u)));
+    const uint32_t mine = warp == 0 ? f0 : (warp == 1 ? f1 : (warp == 2 ? f2 : f3));
     if ((mine >> lane) & 1u) {
       int b = -1;
       uint32_t occ = occurs[i];
@@ -464,7 +491,7 @@ __global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const i
       }
       best[i] = b;
     }
-    __syncthreads();
+    qsync();
     // pair the blocks that name each other; each pair is written by its lower block
     if ((mine >> lane) & 1u) {
       const int b = best[i];
@@ -473,30 +500,30 @@ __global__ void __launch_bounds__(kPairThreads) pair_query_blocks_kernel(const i
         partner[b] = i;
       }
     }
-    __syncthreads();
+    qsync();
     const uint32_t still = __ballot_sync(0xFFFFFFFFu, ((mine >> lane) & 1u) && partner[i] < 0);
-    if (lane == 0 && warp < kPairMaxQB / 32) {
+    if (lane == 0) {
       freew[warp] = still;
       wcnt[warp] = __popc(still);
     }
-    __syncthreads();
+    qsync();
     nfree = wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
   }
   // tile n: the pair (or the lone block) whose lower block is the n-th lowest
   const bool lead = i < NQB && (partner[i] > i || partner[i] == -2);
   const uint32_t bal = __ballot_sync(0xFFFFFFFFu, lead);
-  __syncthreads();  // every thread has read wcnt
-  if (lane == 0 && warp < kPairMaxQB / 32) wcnt[warp] = __popc(bal);
-  __syncthreads();
+  qsync();  // every thread has read wcnt
+  if (lane == 0) wcnt[warp] = __popc(bal);
+  qsync();
   int before = __popc(bal & ((1u << lane) - 1u));
-  for (int w = 0; w < warp && w < kPairMaxQB / 32; ++w) before += wcnt[w];
+  for (int w = 0; w < warp; ++w) before += wcnt[w];
   const int n = wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
   int32_t* out = qpair + (size_t)bh * MT * 2;
   if (lead && before < MT) {
     out[2 * before] = i;
     out[2 * before + 1] = partner[i] >= 0 ? partner[i] : -1;
   }
-  for (int t = n + tid; t < MT; t += kPairThreads) {  // tiles without query blocks (none when MT = ceil(NQB / 2))
+  for (int t = n + tid; t < MT; t += kPairMaxQB) {  // tiles without query blocks (none when MT = ceil(NQB / 2))
     out[2 * t] = -1;
     out[2 * t + 1] = -1;
   }

@@ -166,5 +166,7 @@ int check_chunk_call(const void* q, const void* k, const void* v, const cva_kv_c
 
 // ---- diagnostics (diag.cu) ------------------------------------------------
 cudaError_t launch_wait_timeout(int* err, int* result, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_mma_cycles(int M, int N, int iters, unsigned long long* cycles, int sms, int* err,
+                              cudaStream_t stream);
 
 }  // namespace cva

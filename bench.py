@@ -67,6 +67,9 @@ def parse_args():
     ap.add_argument("--qkv", action="store_true",
                     help="the QKV projection fused with rotation/append/pooling (hidden = H*D) "
                          "against cuBLAS GEMMs followed by the separate kernels (measurement mode)")
+    ap.add_argument("--mma-shapes", action="store_true",
+                    help="tensor-core time of one tcgen05.mma per shape (64- and 128-row tiles), "
+                         "one JSON line each (measurement mode)")
     return ap.parse_args()
 
 
@@ -897,6 +900,27 @@ def run_qkv(args):
     return 0
 
 
+def run_mma_shapes(args):
+    """Cycles per back-to-back tcgen05.mma (bf16, K = 16) for the tile shapes the
+    attention could use, one CTA per SM; the median over the SMs of the
+    second of two runs."""
+    import torch
+    from autoregressive_video_dit_b200 import ops
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device="cuda")
+    iters = 1024
+    for m, n in ((128, 128), (64, 128), (128, 256), (64, 256), (128, 64), (64, 64)):
+        for _ in range(2):
+            ops.diag_mma_cycles(m, n, iters, cycles)
+            torch.cuda.synchronize()
+        assert ops.device_status() == 0
+        per = float(cycles.median().item()) / (4 * iters)
+        print(json.dumps({"mode": "mma shapes", "m": m, "n": n, "k": 16, "cycles_per_mma": per,
+                          "flop_per_cycle_per_sm": 2.0 * m * n * 16 / per, "ctas": sms,
+                          "mmas_per_cta": 4 * iters}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -907,6 +931,8 @@ def main():
         return run_sweep(args)
     if args.stream:
         return run_stream(args)
+    if args.mma_shapes:
+        return run_mma_shapes(args)
     return run_cuda(args)
 
 

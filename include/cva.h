@@ -418,6 +418,20 @@ int cva_set_stage_events(void* const* events, int32_t n);
  * kernel returns normally and the context stays usable. */
 int cva_diag_wait_timeout(int32_t limit_us, int32_t* result, cva_stream_t stream);
 
+/* Diagnostic of the tensor cores: `ctas` CTAs (at most one per SM) each issue
+ * iters x 4 back-to-back tcgen05.mma kind::f16 of shape m x n x 16 (bf16
+ * zeros from shared memory, fp32 accumulator in tensor memory) from one
+ * thread and wait for them (bounded; a timeout latches CVA_DEV_TIMEOUT);
+ * cycles[c] gets CTA c's clock64 span, so cycles / (4 iters) is the time of
+ * one MMA. m: 64 or 128; n: a multiple of 8 (m = 64) or 16 (m = 128) in
+ * [8, 256]; iters in [1, 65536]. cycles: device buffer of ctas uint64
+ * values, 8-byte aligned. It is what shows that a 64-row MMA takes the
+ * tensor time of a 128-row one, which is why attention tiles hold 128 rows
+ * ("Light Forcing" section 2.2 picks per 64-token query block; two blocks
+ * share a tile). */
+int cva_diag_mma_cycles(int32_t m, int32_t n, int32_t iters, uint64_t* cycles, int32_t ctas,
+                        cva_stream_t stream);
+
 /* Chunk budget from the noise level ("Light Forcing", section 2.1: s_i =
  * s_base - alpha_i beta, alpha_i scaling with the noise level as 1/sqrt(T),
  * beta set so that the total FLOPs meet a target sparsity). Readings: alpha_i

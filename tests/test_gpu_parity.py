@@ -837,6 +837,19 @@ def test_bounded_wait_gives_up_and_latches_a_timeout(ops):
     assert float(y.sum()) == 36.0
 
 
+def test_mma_cycle_diagnostic_runs_and_checks_its_arguments(ops):
+    import torch
+    cycles = torch.zeros(4, dtype=torch.int64, device="cuda")
+    ops.diag_mma_cycles(128, 128, 64, cycles)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    per = cycles.cpu().numpy() / (4 * 64)
+    assert (per > 8).all() and (per < 10000).all(), per
+    for m, n in ((96, 128), (128, 24), (64, 4), (128, 512)):
+        with pytest.raises(ops.CvaError):
+            ops.diag_mma_cycles(m, n, 64, cycles)
+
+
 def test_host_errors(ops):
     import torch
     wl = WORKLOADS["r64"]
