@@ -551,6 +551,35 @@ def test_rotate_append_pool_is_the_fused_calls_first_launch(ops, key):
     torch.testing.assert_close(qpool, ref, rtol=1e-6, atol=1e-6)
 
 
+def test_chunk_call_replays_from_a_cuda_graph(ops):
+    # The fused call (rotation, selection, pairing, attention, merge, the later
+    # launches programmatic dependents) captured once into a CUDA graph and
+    # replayed gives the eager call's bits.
+    import torch
+    wl = WORKLOADS["c3"].with_chunk(7)
+    res, cache = _gpu_stream(ops, wl, 7)
+    out_eager, ws, k_f, k_b = res[7]
+    x = inputs(wl, 7, 0, None, key_centres(wl, 0) if wl.keys == "clustered" else None)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    tabs = _tables(ops, wl, 0)
+    out = torch.empty((wl.B, wl.Lq, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        ops.chunk_attention(q, k, v, cache, tabs, wl.t0_of(7), k_f, k_b, ws, out)   # warm-up
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.chunk_attention(q, k, v, cache, tabs, wl.t0_of(7), k_f, k_b, ws, out)
+    for _ in range(3):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(from_dev(out), out_eager)
+    assert ops.device_status() == 0
+
+
 def test_c4_end_to_end_sampled(ops):
     wl = WORKLOADS["c4"]
     heads = [0, 21, 39]
