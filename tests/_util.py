@@ -244,3 +244,23 @@ def rope_tol(y64: np.ndarray) -> np.ndarray:
 
 
 __all__ = [n for n in dir() if not n.startswith("_")] + ["WORKLOADS", "math"]
+
+
+def mutual_best_pairs(frames):
+    """Rounds: every unpaired query block names the unpaired block sharing the
+    most picked frames (31 or more count as equal), ties to the lower index;
+    blocks naming each other pair up; a last lone block pairs with none (-1).
+    Pairs in order of their lower block."""
+    sets = [set(int(t) for t in f) for f in frames]
+    n = len(sets)
+    ov = lambda i, j: min(len(sets[i] & sets[j]), 31)
+    free, partner = set(range(n)), {}
+    while len(free) >= 2:
+        best = {}
+        for i in free:
+            best[i] = max((j for j in free if j != i), key=lambda j: (ov(i, j), -j))
+        for i in free:
+            if best[i] > i and best[best[i]] == i:
+                partner[i], partner[best[i]] = best[i], i
+        free -= set(partner)
+    return [(i, partner[i]) if i in partner else (i, -1) for i in range(n) if partner.get(i, n) > i]

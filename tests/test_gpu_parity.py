@@ -20,7 +20,7 @@ from oracle import rope as o_rope
 
 from _util import (MAX_ABS, MEAN_ABS, attn_errors, bits_to_f64, f64_to_bits, from_dev, inputs,
                    lib_budget, oracle_budget, hist_count, rope_tol, sample_rows, check_selection, ws_lists, oracle_run,
-                   shape_of, to_dev)
+                   shape_of, to_dev, mutual_best_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -452,26 +452,6 @@ def _ws_pairs(wl, ws, k_f, k_b):
     return raw[o_p:o_p + d.B * d.H * MT * 8].view(np.int32).reshape(d.B * d.H, MT, 2)
 
 
-def _mutual_best_pairs(frames):
-    """Rounds: every unpaired query block names the unpaired block sharing the
-    most picked frames (31 or more count as equal), ties to the lower index;
-    blocks naming each other pair up; a last lone block pairs with none (-1).
-    Pairs in order of their lower block."""
-    sets = [set(int(t) for t in f) for f in frames]
-    n = len(sets)
-    ov = lambda i, j: min(len(sets[i] & sets[j]), 31)
-    free, partner = set(range(n)), {}
-    while len(free) >= 2:
-        best = {}
-        for i in free:
-            best[i] = max((j for j in free if j != i), key=lambda j: (ov(i, j), -j))
-        for i in free:
-            if best[i] > i and best[best[i]] == i:
-                partner[i], partner[best[i]] = best[i], i
-        free -= set(partner)
-    return [(i, partner[i]) if i in partner else (i, -1) for i in range(n) if partner.get(i, n) > i]
-
-
 def test_query_block_pairs_are_mutual_best(ops):
     # c3 chunk 7: 18 history frames, 8 picked per query block, so the fused
     # call pairs the 64-row query blocks by shared frames before the attention
@@ -485,7 +465,7 @@ def test_query_block_pairs_are_mutual_best(ops):
     fr = fr.reshape(wl.B * wl.H, wl.NQB, kfe)
     got = _ws_pairs(wl, ws, k_f, k_b)
     for bh in range(wl.B * wl.H):
-        want = _mutual_best_pairs(fr[bh])
+        want = mutual_best_pairs(fr[bh])
         assert [tuple(int(v) for v in p) for p in got[bh, :len(want)]] == want, bh
         assert (got[bh, len(want):] == -1).all()
         ids = sorted(v for p in want for v in p if v >= 0)

@@ -8,7 +8,7 @@ that rule on hand-made scores and on a small oracle run.
 """
 import numpy as np
 
-from _util import check_selection, oracle_budget, valid_topk
+from _util import mutual_best_pairs, check_selection, oracle_budget, valid_topk
 from cva_workload import WORKLOADS, chunk_inputs, bf16_bits_to_f32
 from oracle import path
 
@@ -70,3 +70,35 @@ def test_check_selection_counts_wrong_lists_and_substitutes_valid_ones():
         f2[b, h, qb, 0] = unpicked[0]
         f2[b, h, qb] = np.sort(f2[b, h, qb])
         assert check_selection(run, f2, bl, cnt)[1] >= 1
+
+
+def test_mutual_best_pairs_by_hand():
+    # frame sets of 5 query blocks: 0 and 3 share three frames, 1 and 2 two,
+    # 4 shares at most one with anyone: round 1 pairs (0, 3) and (1, 2); block
+    # 4 is left alone
+    frames = [[0, 1, 2], [5, 6, 7], [5, 6, 9], [0, 1, 2], [2, 9, 11]]
+    assert mutual_best_pairs(frames) == [(0, 3), (1, 2), (4, -1)]
+    # ties go to the lower index: 1, 2 and 3 all share one frame with 0
+    frames = [[0, 1], [0, 5], [0, 6], [0, 7]]
+    assert mutual_best_pairs(frames) == [(0, 1), (2, 3)]
+
+
+def test_mutual_best_pairs_partition_and_round_rule():
+    rng = np.random.default_rng(7)
+    for trial in range(40):
+        n = int(rng.integers(1, 40))
+        F, k = int(rng.integers(2, 20)), None
+        k = int(rng.integers(1, F + 1))
+        frames = [sorted(rng.choice(F, size=k, replace=False).tolist()) for _ in range(n)]
+        pairs = mutual_best_pairs(frames)
+        ids = sorted(v for p in pairs for v in p if v >= 0)
+        assert ids == list(range(n))                              # a partition
+        assert [p[0] for p in pairs] == sorted(p[0] for p in pairs)
+        assert all(j == -1 or i < j for i, j in pairs)
+        assert sum(1 for _, j in pairs if j == -1) == n % 2     # one lone block at most
+        # the best pair overall (most shared frames, then lowest indices) is always formed
+        if n >= 2:
+            sets = [set(f) for f in frames]
+            ov = lambda i, j: min(len(sets[i] & sets[j]), 31)
+            top = max(((ov(i, j), -i, -j) for i in range(n) for j in range(i + 1, n)))
+            assert (-top[1], -top[2]) in pairs
